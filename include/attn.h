@@ -1,0 +1,158 @@
+/*
+ * attn.h - C ABI of libattn: exact blockwise self-attention forward on NVIDIA B200
+ * (sm_100a), and the merge of partial results.
+ *
+ * What is computed. For every batch b, query head h and query row i:
+ *     s_j   = scale * <q[b,h,i,:], k[b,g,j,:]>   over the visible keys j,
+ *     O_i   = sum_j softmax(s)_j * v[b,g,j,:],
+ *     LSE_i = ln(sum_j exp(s_j)),
+ * with g = h / (Hq / Hkv). This is the conventional three-step attention
+ * ("FlashAttention by hand": logits, a softmax row that sums to one, weights times
+ * values), reached exactly, up to floating-point rounding, by the tiled online
+ * softmax the same page describes: key/value tiles streamed through on-chip
+ * memory, a running maximum and denominator, rescaling of the partial output when
+ * the maximum grows, and one final division. The score matrix never reaches
+ * global memory.
+ *
+ * Masking. With causal != 0, key j is visible to query i when
+ * kv_off + j <= q_off + i (global positions; HOF SWIFT Attention, section 3,
+ * Transform stage names causal masking). A row with no visible key has O = 0 and
+ * LSE = -inf.
+ *
+ * Layouts. q, k, v are bf16, row-major [B][H][N][d] (d contiguous). O is fp32
+ * [B][Hq][Nq][d]; LSE is fp32 [B][Hq][Nq], natural log, scale included.
+ *
+ * Ownership and execution. The caller owns every buffer; the library allocates no
+ * device memory. All pointers named "device" must be device (or managed) memory.
+ * Calls enqueue work on `stream` (a cudaStream_t; NULL is the legacy default
+ * stream) and return without waiting. Buffers must stay valid until that work has
+ * finished. No call throws; every call returns an attn_status_t.
+ *
+ * Errors. Arguments are checked before anything is launched: null or misaligned
+ * pointers, non-positive sizes, Hq not a multiple of Hkv, outputs overlapping
+ * inputs, a negative or non-finite scale, and offsets/leading dimensions that do
+ * not fit give ATTN_ERR_INVALID_ARG. Shapes the kernels are not built for (d other
+ * than 64 or 128, more than ATTN_MAX_MERGE_PARTS parts, sizes beyond the tensor-map
+ * limits) give ATTN_ERR_UNSUPPORTED. A failed CUDA call gives ATTN_ERR_CUDA. A
+ * device-side wait that ran out of time is reported by attn_device_status as
+ * ATTN_ERR_TIMEOUT; it never traps. NaN or Inf inside q, k, v is not checked and
+ * gives unspecified results.
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,
+  ATTN_ERR_UNSUPPORTED = 2,
+  ATTN_ERR_CUDA = 3,
+  ATTN_ERR_TIMEOUT = 4,
+  ATTN_ERR_INJECTED = 5
+} attn_status_t;
+
+#define ATTN_MAX_MERGE_PARTS 64
+
+/* Static description of a status code. Never NULL. */
+const char* attn_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+int attn_version(void);
+
+/*
+ * attn_fwd - single-pass attention over a whole sequence ("FlashAttention by hand",
+ * paragraphs on the fused tiled computation, the running statistics, rescaling and
+ * the final division).
+ *
+ *   q      device, bf16 [B][Hq][N][d], 16-byte aligned
+ *   k, v   device, bf16 [B][Hkv][N][d], 16-byte aligned
+ *   o      device, fp32 [B][Hq][N][d], 16-byte aligned (written)
+ *   lse    device, fp32 [B][Hq][N], 4-byte aligned (written)
+ *   B, Hq, Hkv >= 1 with Hq % Hkv == 0; N >= 1; d in {64, 128}
+ *   causal 0 or 1 (key j visible to query i iff j <= i)
+ *   scale  finite, >= 0 (normally 1/sqrt(d))
+ *   stream cudaStream_t to enqueue on
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, float* o, float* lse,
+                       int B, int Hq, int Hkv, int64_t N, int d, int causal, float scale,
+                       void* stream);
+
+/*
+ * attn_fwd_partial - attention of one query chunk against one key/value chunk: one
+ * ring step of Ring Attention ("Ring Attention with Blockwise Parallel
+ * Transformers", section 3: each device attends its query block to the key/value
+ * block it currently holds), or one fragment of the ATTENTION2D query x key/value
+ * grid (section 3: fragment-local statistics). The result is the NORMALISED
+ * partial output over this chunk's visible keys plus its LSE, ready for
+ * attn_merge.
+ *
+ *   q        device, bf16: &Q[0][0][q_start][0] of a parent tensor
+ *            [B][Hq][q_ld][d]; the chunk is rows [q_start, q_start + Nq)
+ *   k_chunk, v_chunk
+ *            device, bf16: &K[0][0][kv_start][0] of parents [B][Hkv][kv_ld][d];
+ *            the chunk is rows [kv_start, kv_start + Nkv); rows beyond it are
+ *            never read
+ *   o_part   device, fp32 dense [B][Hq][Nq][d] (written)
+ *   lse_part device, fp32 dense [B][Hq][Nq] (written)
+ *   q_ld >= Nq, kv_ld >= Nkv: allocated sequence length of the parents
+ *   q_off, kv_off >= 0: global position of the chunks' first rows (used only for
+ *            the causal test kv_off + j <= q_off + i)
+ *   other arguments as for attn_fwd. All pointers 16-byte aligned (lse_part 4).
+ */
+attn_status_t attn_fwd_partial(const void* q, const void* k_chunk, const void* v_chunk,
+                               float* o_part, float* lse_part, int B, int Hq, int Hkv,
+                               int64_t Nq, int64_t Nkv, int64_t q_ld, int64_t kv_ld,
+                               int64_t q_off, int64_t kv_off, int d, int causal,
+                               float scale, void* stream);
+
+/*
+ * attn_merge - combine partial results computed over disjoint key sets
+ * (ATTENTION2D, section 3: fragment-local statistics normalised and summed in
+ * stages; section 2: the combination is commutative and associative, so no
+ * approximation enters). Per row, with M = max_i LSE_i and w_i = exp(LSE_i - M):
+ *     O = sum_i w_i O_i / sum_i w_i,   LSE = M + ln(sum_i w_i).
+ * Parts with LSE = -inf contribute nothing; if all are -inf, O = 0, LSE = -inf.
+ * n_parts = 1 copies. The result does not depend on the order of the parts beyond
+ * fp32 rounding.
+ *
+ *   o_parts, lse_parts  HOST arrays of n_parts DEVICE pointers: fp32 [rows][d]
+ *                       (16-byte aligned) and fp32 [rows] (4-byte aligned)
+ *   n_parts             1 .. ATTN_MAX_MERGE_PARTS
+ *   o, lse              device, fp32 [rows][d] and [rows] (written); must not
+ *                       overlap any part
+ *   rows >= 1; d in {64, 128}
+ */
+attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_parts,
+                         int n_parts, float* o, float* lse, int64_t rows, int d,
+                         void* stream);
+
+/*
+ * attn_device_status - synchronise `stream` and report whether any kernel of this
+ * library on the current device recorded a device-side failure since the last
+ * reset (ATTN_ERR_TIMEOUT: a bounded wait ran out; the kernel then stopped its
+ * work and returned, leaving its outputs unspecified). reset != 0 clears the
+ * record. Returns ATTN_ERR_CUDA if synchronising fails.
+ */
+attn_status_t attn_device_status(void* stream, int reset);
+
+/*
+ * attn_debug_inject - host-side fault injection for tests of error paths: the next
+ * `count` calls of attn_fwd, attn_fwd_partial or attn_merge return `status`
+ * (which must be a failure code) after argument checks and before any launch.
+ * count = 0 disarms. Not thread-safe; for tests only.
+ */
+attn_status_t attn_debug_inject(int status, int count);
+
+/* Number of CUDA kernels this library has launched in this process (all devices). */
+uint64_t attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */

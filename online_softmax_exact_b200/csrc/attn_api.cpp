@@ -1,0 +1,166 @@
+// attn_api.cpp - the C ABI of libattn: argument checks, fault injection for tests, and
+// dispatch to the launchers. Every check here runs before any CUDA call, so invalid
+// arguments are reported without touching a device.
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/attn.h"
+#include "attn_internal.h"
+
+namespace {
+
+int g_inject_status = ATTN_OK;
+int g_inject_count = 0;
+
+// Largest chunk length: TMA row coordinates are 32-bit and a unit reaches 256 rows past
+// its start.
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 512;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Span {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+Span span(const void* p, uint64_t bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return Span{lo, lo + static_cast<uintptr_t>(bytes)};
+}
+
+bool overlap(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi; }
+
+attn_status_t take_injected() {
+  if (g_inject_count > 0) {
+    --g_inject_count;
+    return static_cast<attn_status_t>(g_inject_status);
+  }
+  return ATTN_OK;
+}
+
+attn_status_t check_and_launch(const void* q, const void* k, const void* v, float* o, float* lse,
+                               int B, int Hq, int Hkv, int64_t Nq, int64_t Nkv, int64_t q_ld,
+                               int64_t kv_ld, int64_t q_off, int64_t kv_off, int d, int causal,
+                               float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (Nq < 1 || Nkv < 1 || q_ld < Nq || kv_ld < Nkv || q_off < 0 || kv_off < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Nq > kMaxRows || Nkv > kMaxRows || q_ld > kMaxRows || kv_ld > kMaxRows)
+    return ATTN_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hq > (int64_t(1) << 30) || q_off > (int64_t(1) << 60) ||
+      kv_off > (int64_t(1) << 60))
+    return ATTN_ERR_UNSUPPORTED;
+
+  const uint64_t bh = (uint64_t)B * Hq, bhkv = (uint64_t)B * Hkv;
+  const Span sq = span(q, ((bh - 1) * q_ld + Nq) * d * 2);
+  const Span sk = span(k, ((bhkv - 1) * kv_ld + Nkv) * d * 2);
+  const Span sv = span(v, ((bhkv - 1) * kv_ld + Nkv) * d * 2);
+  const Span so = span(o, bh * Nq * d * 4);
+  const Span sl = span(lse, bh * Nq * 4);
+  if (overlap(so, sq) || overlap(so, sk) || overlap(so, sv) || overlap(sl, sq) ||
+      overlap(sl, sk) || overlap(sl, sv) || overlap(so, sl))
+    return ATTN_ERR_INVALID_ARG;
+
+  attn_status_t inj = take_injected();
+  if (inj != ATTN_OK) return inj;
+
+  osx::FwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.q_ld = q_ld;
+  a.kv_ld = kv_ld;
+  a.q_off = q_off;
+  a.kv_off = kv_off;
+  a.d = d;
+  a.causal = causal;
+  a.scale = scale;
+  return static_cast<attn_status_t>(osx::launch_fwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK: success";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG: invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED: shape or size not supported";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT: a device-side wait ran out of time";
+    case ATTN_ERR_INJECTED: return "ATTN_ERR_INJECTED: failure injected by attn_debug_inject";
+    default: return "unknown attn status";
+  }
+}
+
+int attn_version(void) { return (1 << 16) | 0; }
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, float* o, float* lse, int B,
+                       int Hq, int Hkv, int64_t N, int d, int causal, float scale, void* stream) {
+  return check_and_launch(q, k, v, o, lse, B, Hq, Hkv, N, N, N, N, 0, 0, d, causal, scale, stream);
+}
+
+attn_status_t attn_fwd_partial(const void* q, const void* k_chunk, const void* v_chunk,
+                               float* o_part, float* lse_part, int B, int Hq, int Hkv, int64_t Nq,
+                               int64_t Nkv, int64_t q_ld, int64_t kv_ld, int64_t q_off,
+                               int64_t kv_off, int d, int causal, float scale, void* stream) {
+  return check_and_launch(q, k_chunk, v_chunk, o_part, lse_part, B, Hq, Hkv, Nq, Nkv, q_ld, kv_ld,
+                          q_off, kv_off, d, causal, scale, stream);
+}
+
+attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts,
+                         float* o, float* lse, int64_t rows, int d, void* stream) {
+  if (!o_parts || !lse_parts || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (n_parts < 1 || rows < 1) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(lse, 4)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (n_parts > ATTN_MAX_MERGE_PARTS) return ATTN_ERR_UNSUPPORTED;
+  if (rows > (int64_t(1) << 40)) return ATTN_ERR_UNSUPPORTED;
+  const Span so = span(o, (uint64_t)rows * d * 4);
+  const Span sl = span(lse, (uint64_t)rows * 4);
+  if (overlap(so, sl)) return ATTN_ERR_INVALID_ARG;
+  for (int i = 0; i < n_parts; ++i) {
+    if (!o_parts[i] || !lse_parts[i]) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(o_parts[i], 16) || !aligned(lse_parts[i], 4)) return ATTN_ERR_INVALID_ARG;
+    const Span po = span(o_parts[i], (uint64_t)rows * d * 4);
+    const Span pl = span(lse_parts[i], (uint64_t)rows * 4);
+    if (overlap(so, po) || overlap(so, pl) || overlap(sl, po) || overlap(sl, pl))
+      return ATTN_ERR_INVALID_ARG;
+  }
+  attn_status_t inj = take_injected();
+  if (inj != ATTN_OK) return inj;
+  return static_cast<attn_status_t>(osx::launch_merge(o_parts, lse_parts, n_parts, o, lse, rows, d,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
+attn_status_t attn_device_status(void* stream, int reset) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned st = 0;
+  if (osx::read_device_status(&st, reset) != ATTN_OK) return ATTN_ERR_CUDA;
+  return st ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+attn_status_t attn_debug_inject(int status, int count) {
+  if (count < 0) return ATTN_ERR_INVALID_ARG;
+  if (count > 0 && (status <= ATTN_OK || status > ATTN_ERR_INJECTED)) return ATTN_ERR_INVALID_ARG;
+  g_inject_status = status;
+  g_inject_count = count;
+  return ATTN_OK;
+}
+
+uint64_t attn_launch_count(void) { return osx::launch_count(); }
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// attn_kernels.cu - the library's only device translation unit: kernel instantiations,
+// per-device set-up, and launchers.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_fwd_kernel.cuh"
+#include "attn_internal.h"
+#include "attn_merge_kernel.cuh"
+#include "tma_host.h"
+
+namespace osx {
+
+// Device status word (one per device that loads the library): bounded waits that run
+// out record kDevTimeout here. Read through read_device_status().
+__device__ unsigned g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned* status = nullptr;  // device address of g_device_status
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+std::atomic<uint64_t> g_launches{0};
+
+// Per-device set-up, once per device with that device current: SM count, the device
+// address of the status word, and the dynamic shared-memory opt-in of each kernel.
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!di.ready) {
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      void* st = nullptr;
+      if (cudaGetSymbolAddress(&st, g_device_status) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)FwdCfg<64>::kSmemBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)FwdCfg<128>::kSmemBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      di.num_sms = sms;
+      di.status = static_cast<unsigned*>(st);
+      di.ready = true;
+    }
+  }
+  *out = &di;
+  return ATTN_OK;
+}
+
+template <int D>
+int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_rows_bf16(&tq, a.q, (uint64_t)a.B * a.Hq, a.Nq, a.q_ld, D, 128) ||
+      !encode_rows_bf16(&tk, a.k, (uint64_t)a.B * a.Hkv, a.Nkv, a.kv_ld, D, 128) ||
+      !encode_rows_bf16(&tv, a.v, (uint64_t)a.B * a.Hkv, a.Nkv, a.kv_ld, D, 128))
+    return ATTN_ERR_UNSUPPORTED;
+  FwdParams p;
+  p.o = a.o;
+  p.lse = a.lse;
+  p.status = di.status;
+  p.Nq = a.Nq;
+  p.Nkv = a.Nkv;
+  p.q_off = a.q_off;
+  p.kv_off = a.kv_off;
+  p.BH = a.B * a.Hq;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.group = a.Hq / a.Hkv;
+  p.causal = a.causal;
+  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
+  p.n_qpairs = static_cast<int>((a.Nq + 255) / 256);
+  const long long units = (long long)p.n_qpairs * p.BH;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  p.n_units = static_cast<int>(units);
+  p.n_kv_tiles = static_cast<int>((a.Nkv + 127) / 128);
+  const int grid = p.n_units < di.num_sms ? p.n_units : di.num_sms;
+  attn_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return ATTN_OK;
+}
+
+template <int D>
+int launch_merge_d(const MergeParams& p, const DeviceInfo& di, cudaStream_t stream) {
+  constexpr int rpb = 256 / (D / 4);
+  long long blocks = (p.rows + rpb - 1) / rpb;
+  const long long cap = (long long)di.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  attn_merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return ATTN_OK;
+}
+
+}  // namespace
+
+int launch_fwd(const FwdLaunch& a, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != ATTN_OK) return rc;
+  switch (a.d) {
+    case 64: return launch_fwd_d<64>(a, *di, stream);
+    case 128: return launch_fwd_d<128>(a, *di, stream);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+int launch_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts,
+                 float* o, float* lse, long long rows, int d, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != ATTN_OK) return rc;
+  MergeParams p;
+  for (int i = 0; i < kMaxMergeParts; ++i) {
+    p.o[i] = i < n_parts ? o_parts[i] : nullptr;
+    p.lse[i] = i < n_parts ? lse_parts[i] : nullptr;
+  }
+  p.out_o = o;
+  p.out_lse = lse;
+  p.rows = rows;
+  p.n = n_parts;
+  switch (d) {
+    case 64: return launch_merge_d<64>(p, *di, stream);
+    case 128: return launch_merge_d<128>(p, *di, stream);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+int read_device_status(unsigned* out, int reset) {
+  if (cudaMemcpyFromSymbol(out, g_device_status, sizeof(unsigned)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (reset) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(unsigned)) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
+
+}  // namespace osx

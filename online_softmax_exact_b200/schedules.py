@@ -1,0 +1,136 @@
+"""Chunk schedules of the sequence-parallel methods, emulated on one GPU over the C ABI.
+
+Both schedules split the sequence into chunks, run ``attn_fwd_partial`` on (query
+chunk, key/value chunk) pairs and combine each query chunk's partials with
+``attn_merge``. Outputs are chunk-major: O ``[P, B, Hq, C, d]`` and LSE
+``[P, B, Hq, C]`` for P chunks of C rows, i.e. the layout in which chunk i's result
+lives on device i of the distributed method; ``chunks_to_sequence`` gives the
+``[B, Hq, N, d]`` view when wanted.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import attn_fwd_partial, attn_merge
+
+
+def chunk_bounds(N: int, n_chunks: int) -> list[tuple[int, int]]:
+    if n_chunks < 1 or N % n_chunks:
+        raise ValueError("the sequence length must split into equal chunks")
+    c = N // n_chunks
+    return [(i * c, (i + 1) * c) for i in range(n_chunks)]
+
+
+def ring_order(n_chunks: int, causal: bool) -> list[list[int]]:
+    """Key/value chunks each query chunk visits, in ring order: at step s, query chunk
+    i holds key/value chunk (i - s) mod P ("Ring Attention with Blockwise Parallel
+    Transformers", section 3: blocks pass around the ring, one hop per step). Under the
+    causal mask a key/value chunk entirely after the query chunk is hidden and skipped.
+    """
+    out = []
+    for qi in range(n_chunks):
+        visit = []
+        for s in range(n_chunks):
+            kv = (qi - s) % n_chunks
+            if causal and kv > qi:
+                continue
+            visit.append(kv)
+        out.append(visit)
+    return out
+
+
+@dataclass
+class Workspace:
+    """Partial-result buffers reused across calls (one per (query chunk, step))."""
+
+    o: torch.Tensor    # [S, B, Hq, C, d]
+    lse: torch.Tensor  # [S, B, Hq, C]
+
+    @staticmethod
+    def for_shape(slots: int, B: int, Hq: int, C: int, d: int, device) -> "Workspace":
+        return Workspace(torch.empty((slots, B, Hq, C, d), dtype=torch.float32, device=device),
+                         torch.empty((slots, B, Hq, C), dtype=torch.float32, device=device))
+
+
+def _alloc_out(q, n_chunks, out):
+    B, Hq, N, d = q.shape
+    C = N // n_chunks
+    if out is None:
+        return (torch.empty((n_chunks, B, Hq, C, d), dtype=torch.float32, device=q.device),
+                torch.empty((n_chunks, B, Hq, C), dtype=torch.float32, device=q.device))
+    return out
+
+
+def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None = None,
+                   out=None, workspace: Workspace | None = None, stream=None):
+    """Ring Attention's schedule on one GPU: query chunk i attends the key/value chunks
+    of :func:`ring_order` one ring step at a time, then merges its partials.
+
+    Returns chunk-major (O [P,B,Hq,C,d], LSE [P,B,Hq,C]).
+    """
+    B, Hq, N, d = q.shape
+    bounds = chunk_bounds(N, n_chunks)
+    C = N // n_chunks
+    order = ring_order(n_chunks, causal)
+    o_out, l_out = _alloc_out(q, n_chunks, out)
+    slots = max(len(x) for x in order)
+    if workspace is None or workspace.o.shape[0] < slots or workspace.o.shape[1:] != (B, Hq, C, d):
+        workspace = Workspace.for_shape(slots, B, Hq, C, d, q.device)
+    for qi, visit in enumerate(order):
+        qs, qe = bounds[qi]
+        if len(visit) == 1:
+            # one part: the merge is the identity, so write the result in place
+            ks, ke = bounds[visit[0]]
+            attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                             causal=causal, scale=scale, o=o_out[qi], lse=l_out[qi], stream=stream)
+            continue
+        for slot, kv in enumerate(visit):
+            ks, ke = bounds[kv]
+            attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                             causal=causal, scale=scale, o=workspace.o[slot],
+                             lse=workspace.lse[slot], stream=stream)
+        n = len(visit)
+        attn_merge([workspace.o[i] for i in range(n)], [workspace.lse[i] for i in range(n)],
+                   o=o_out[qi], lse=l_out[qi], stream=stream)
+    return o_out, l_out
+
+
+def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], causal: bool,
+                     scale: float | None = None, out=None, workspace: Workspace | None = None,
+                     stream=None):
+    """ATTENTION2D's query x key/value grid on one GPU: every (query chunk, key/value
+    chunk) cell is a partial attention (fragment-local statistics, section 3); each
+    query chunk's partials are merged in the order ``merge_orders[i]`` (any order gives
+    the same result, section 2). Returns chunk-major (O, LSE).
+    """
+    B, Hq, N, d = q.shape
+    bounds = chunk_bounds(N, n_chunks)
+    C = N // n_chunks
+    o_out, l_out = _alloc_out(q, n_chunks, out)
+    if workspace is None or workspace.o.shape[0] < n_chunks or \
+            workspace.o.shape[1:] != (B, Hq, C, d):
+        workspace = Workspace.for_shape(n_chunks, B, Hq, C, d, q.device)
+    for qi in range(n_chunks):
+        qs, qe = bounds[qi]
+        order = merge_orders[qi]
+        if sorted(order) != list(range(n_chunks)):
+            raise ValueError("each merge order must be a permutation of the chunk indices")
+        for kv in range(n_chunks):
+            ks, ke = bounds[kv]
+            attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                             causal=causal, scale=scale, o=workspace.o[kv], lse=workspace.lse[kv],
+                             stream=stream)
+        attn_merge([workspace.o[i] for i in order], [workspace.lse[i] for i in order],
+                   o=o_out[qi], lse=l_out[qi], stream=stream)
+    return o_out, l_out
+
+
+def chunks_to_sequence(o_chunks: torch.Tensor, lse_chunks: torch.Tensor):
+    """[P,B,Hq,C,d] / [P,B,Hq,C] -> [B,Hq,P*C,d] / [B,Hq,P*C] (a copy)."""
+    P, B, Hq, C, d = o_chunks.shape
+    o = o_chunks.permute(1, 2, 0, 3, 4).reshape(B, Hq, P * C, d)
+    lse = lse_chunks.permute(1, 2, 0, 3).reshape(B, Hq, P * C)
+    return o, lse
