@@ -1,0 +1,531 @@
+"""Benchmark of exact blockwise attention forward + (O, LSE) merge on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload ring_32k]
+
+One step is one pass of the whole path over one batch of synthetic input: for the
+default workload (B=1, H=32, N=32768, d=128, causal, Ring Attention's schedule of 8
+query/key-value chunks emulated on one GPU) that is 36 partial attentions and 7
+merges. The line printed by rank 0 reports:
+
+  value      device-timed TFLOP/s of the whole job (nominal causal FLOPs
+             4*B*H*N^2*d/2 per step, summed over ranks, over the max-over-ranks time),
+             inputs resident in HBM; inputs (768 MiB) exceed L2, so no flush is needed;
+  roofline   the attention kernel's achieved TFLOP/s (algorithmic FLOPs per launch over
+             its CUDA-event duration, on its stream) against the measured bf16 peak;
+  merge      the merge kernel's achieved GB/s against the measured HBM copy bandwidth;
+  e2e        the same metric through the public API with pinned host buffers: the
+             host->device copies of Q, K, V and the device->host copy of O, LSE are
+             inside the timed region;
+  cpu_baseline  the fp64 oracle on the host cores, on a bounded row sample of the
+             same workload (rank 0, N=1 only).
+
+With --gpus N > 1 (launched by torchrun), every rank runs its own independent
+problem of the same size (different seed): weak scaling, no data-path collective.
+``--impl reference`` times the fp64 oracle on the host cores instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------------------
+# host-side helpers (no GPU needed; covered by tests/test_bench_host.py)
+# --------------------------------------------------------------------------------------
+def dist_env() -> tuple[int, int, int]:
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Independent problem per rank: same shapes, different seeded inputs."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(n: int, device) -> int:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return int(n)
+    t = torch.tensor([n], dtype=torch.int64, device=device)
+    dist.all_reduce(t)
+    return int(t.item())
+
+
+def load_peaks() -> tuple[dict, str]:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            d = json.loads(p.read_text())
+            return d, "measured"
+        except Exception:
+            pass
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ring_step_plan(n_chunks: int, causal: bool):
+    """(partial launches with their nominal FLOP fraction of a full chunk pair, merges
+    with their part counts) of one ring step."""
+    from online_softmax_exact_b200.schedules import ring_order
+
+    order = ring_order(n_chunks, causal)
+    partial_fracs, merge_parts = [], []
+    for qi, visit in enumerate(order):
+        for kv in visit:
+            partial_fracs.append(0.5 if (causal and kv == qi) else 1.0)
+        if len(visit) > 1:
+            merge_parts.append(len(visit))
+    return partial_fracs, merge_parts
+
+
+def merge_bytes(n_parts: int, rows: int, d: int) -> int:
+    """Algorithmic HBM bytes of one merge: each part's O and LSE read once, the result
+    written once (fp32)."""
+    return (n_parts + 1) * rows * (d + 1) * 4
+
+
+def parse_clocks(csv_text: str, bus_id: str | None = None) -> dict:
+    """Summarise nvidia-smi samples: median SM clock under load and active reasons."""
+    lines = [ln.strip() for ln in csv_text.strip().splitlines() if ln.strip()]
+    if len(lines) < 2:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    header = [h.strip() for h in lines[0].split(",")]
+    rows = [[c.strip() for c in ln.split(",")] for ln in lines[1:] if not ln.startswith(header[0])]
+
+    def col(name):
+        for i, h in enumerate(header):
+            if h.startswith(name):
+                return i
+        return None
+
+    i_bus, i_sm, i_max = col("pci.bus_id"), col("clocks.current.sm"), col("clocks.max.sm")
+    i_pw = col("power.draw")
+    flags = {"hw_slowdown": col("clocks_event_reasons.hw_slowdown"),
+             "hw_thermal_slowdown": col("clocks_event_reasons.hw_thermal_slowdown"),
+             "sw_thermal_slowdown": col("clocks_event_reasons.sw_thermal_slowdown"),
+             "sw_power_cap": col("clocks_event_reasons.sw_power_cap")}
+    sel = []
+    for r in rows:
+        if len(r) != len(header):
+            continue
+        if bus_id and i_bus is not None and not r[i_bus].upper().startswith(bus_id.upper()):
+            continue
+        sel.append(r)
+
+    def num(s):
+        try:
+            return float(s.split()[0])
+        except Exception:
+            return None
+
+    sm = [num(r[i_sm]) for r in sel if i_sm is not None and num(r[i_sm]) is not None]
+    mx = [num(r[i_max]) for r in sel if i_max is not None and num(r[i_max]) is not None]
+    pw = [num(r[i_pw]) for r in sel if i_pw is not None and num(r[i_pw]) is not None]
+    # "under load": samples drawing well above idle power, else all samples
+    load = [s for s, p in zip(sm, pw) if p is not None and p > 300.0] if pw else []
+    use = load or sm
+    reasons = sorted({name for r in sel for name, i in flags.items()
+                      if i is not None and r[i].lower().startswith("active")})
+    return {"sm_mhz": statistics.median(use) if use else None,
+            "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(sel),
+            "samples_under_load": len(load)}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of clocks and throttle reasons while the timed region runs."""
+
+    QUERY = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.tmp = None
+
+    def __enter__(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self) -> dict:
+        if self.proc is None or self.tmp is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.tmp.flush()
+        text = Path(self.tmp.name).read_text()
+        try:
+            os.unlink(self.tmp.name)
+        except OSError:
+            pass
+        return parse_clocks(text, self.bus_id)
+
+
+# --------------------------------------------------------------------------------------
+# oracle baseline (rank 0 only)
+# --------------------------------------------------------------------------------------
+def oracle_sample_throughput(w, seconds: float, seed: int = 0) -> dict:
+    """Time the fp64 oracle on rows of the workload until ~``seconds`` of CPU work:
+    returns nominal TFLOP/s (4 * visible keys * d per row), rows and threads used."""
+    import numpy as np
+
+    import oracle
+    from workloads import attention_inputs
+
+    q, k, v = attention_inputs(w)
+    rng = np.random.default_rng(seed)
+    threads = oracle.default_threads()
+    flops = 0.0
+    rows_done = 0
+    t_total = 0.0
+    batch = 16
+    while t_total < seconds:
+        rows = np.sort(rng.choice(w.N, size=batch, replace=False)).astype(np.int64)
+        b = int(rng.integers(0, w.B))
+        h = int(rng.integers(0, w.Hq))
+        g = h // (w.Hq // w.Hkv)
+        qh = q[b:b + 1, h:h + 1]
+        kh, vh = k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
+        t0 = time.perf_counter()
+        oracle.attention_rows(qh, kh, vh, causal=w.causal, scale=w.scale, rows=rows)
+        t_total += time.perf_counter() - t0
+        vis = (rows + 1) if w.causal else np.full(batch, w.N)
+        flops += float(4.0 * vis.sum() * w.d)
+        rows_done += batch
+        batch = min(batch * 2, 512)
+    return {"tflops": flops / t_total / 1e12, "rows": rows_done, "seconds": t_total,
+            "threads": threads, "flops": flops}
+
+
+def run_reference(args, w) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    oracle.build()
+    per_step = args.cpu_seconds if args.cpu_seconds_set else \
+        max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_throughput(w, per_step / 4)
+    vals, rows, secs, threads = [], 0, 0.0, 1
+    flops = 0.0
+    for s in range(args.steps):
+        r = oracle_sample_throughput(w, per_step, seed=s + 1)
+        vals.append(r["tflops"])
+        rows += r["rows"]
+        secs += r["seconds"]
+        flops += r["flops"]
+        threads = r["threads"]
+    value = flops / secs / 1e12
+    sample = (f"{rows} query rows of {w.name} drawn uniformly over (batch, head, row), "
+              f"each row's full softmax materialised; {per_step:.1f} s of CPU work per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.flops / (value * 1e12) if value > 0 else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "note": "fp64 CPU oracle (plain materialised softmax, OpenMP over rows); "
+                "ms_per_step is extrapolated from the sampled rows' throughput",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------------------
+METRIC = "attention fwd TFLOP/s and % of bf16 tensor peak on 1 B200; merge HBM GB/s"
+
+
+def workload_config(w, world: int) -> dict:
+    return {"workload": f"{w.name}: {w.description}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+            "N": w.N, "d": w.d, "causal": w.causal, "schedule": w.schedule,
+            "n_chunks": w.n_chunks, "global_batch": w.B * world, "seq_len": w.N,
+            "parallelism": "single GPU" if world == 1 else f"{world} independent replicas",
+            "l2": "inputs larger than L2 (Q, K, V = 768 MiB per step); no flush"}
+
+
+class EventTimer:
+    """Brackets launches with CUDA events on the launching stream."""
+
+    def __init__(self, stream):
+        self.stream = stream
+        self.records = []  # (kind, start, end)
+        self.enabled = False
+        self._kind = None
+
+    def __call__(self, kind: str):
+        self._kind = kind
+        return self
+
+    def __enter__(self):
+        if self.enabled:
+            import torch
+
+            self._s = torch.cuda.Event(enable_timing=True)
+            self._s.record(self.stream)
+        return self
+
+    def __exit__(self, *exc):
+        if self.enabled:
+            import torch
+
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(self.stream)
+            self.records.append((self._kind, self._s, e))
+        return False
+
+    def totals(self) -> dict:
+        out = {}
+        for kind, s, e in self.records:
+            t, n = out.get(kind, (0.0, 0))
+            out[kind] = (t + s.elapsed_time(e), n + 1)
+        return out
+
+
+def run_ours(args, w) -> int:
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    import online_softmax_exact_b200 as osx
+    from online_softmax_exact_b200.schedules import Workspace, ring_attention
+    from workloads import attention_inputs
+    from workloads.configs import Workload
+
+    wr = Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})
+    q_h, k_h, v_h = attention_inputs(wr)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    B, Hq, N, d = q.shape
+    P, C = w.n_chunks, w.N // w.n_chunks
+    out = (torch.empty((P, B, Hq, C, d), dtype=torch.float32, device=dev),
+           torch.empty((P, B, Hq, C), dtype=torch.float32, device=dev))
+    ws = Workspace.for_shape(P, B, Hq, C, d, dev)
+    stream = torch.cuda.current_stream(dev)
+    timer = EventTimer(stream)
+
+    def step():
+        ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
+                       workspace=ws, stream=stream, timer=timer)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if osx.attn_device_status(reset=True) != osx.ATTN_OK:
+        raise RuntimeError("device-side wait ran out of time during warm-up")
+
+    try:
+        pr = torch.cuda.get_device_properties(dev)
+        bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}"
+    except Exception:
+        bus = None
+    n0 = osx.attn_launch_count()
+    timer.enabled = True
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(bus) as clocks:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    timer.enabled = False
+    launches = osx.attn_launch_count() - n0
+    ms = t0.elapsed_time(t1)
+    if osx.attn_device_status() != osx.ATTN_OK:
+        raise RuntimeError("device-side wait ran out of time in the timed region")
+    tot = timer.totals()
+    clk = clocks.summary()
+
+    ms_max = max_over_ranks(ms, dev)
+    launches = sum_over_ranks(launches, dev)
+
+    # ---- per-kernel roofline (this rank's events)
+    peaks, peak_src = load_peaks()
+    fracs, merges = ring_step_plan(P, w.causal)
+    full_pair_flops = 4.0 * B * Hq * C * C * d
+    partial_flops_per_step = full_pair_flops * sum(fracs)
+    t_part, n_part = tot.get("partial", (0.0, 0))
+    t_merge, n_merge = tot.get("merge", (0.0, 0))
+    attn_achieved = partial_flops_per_step * args.steps / (t_part * 1e-3) / 1e12
+    rows = B * Hq * C
+    mbytes = sum(merge_bytes(n, rows, d) for n in merges) * args.steps
+    merge_gbs = mbytes / (t_merge * 1e-3) / 1e9 if t_merge > 0 else None
+    peak_t = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    peak_h = peaks.get("hbm_gbs")
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = run_e2e(args, w, q_h, k_h, v_h, dev, out, ws, world)
+
+    total_flops = w.flops * args.steps * world
+    value = total_flops / (ms_max * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: bf16 N(0,1) from a seeded torch CPU generator",
+        "config": workload_config(w, world),
+        "pct_of_bf16_peak": 100.0 * (value / world) / peak_t,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128> (attn_fwd_partial)",
+                     "achieved": attn_achieved, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": attn_achieved / peak_t,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a "
+                                    f"long back-to-back loop)",
+                     "traffic": None,
+                     "launches": n_part, "avg_launch_ms": t_part / max(1, n_part)},
+        "merge": {"bound": "hbm", "kernel": "attn_merge_kernel<128>", "achieved": merge_gbs,
+                  "peak": peak_h, "unit": "GB/s",
+                  "frac": (merge_gbs / peak_h) if merge_gbs else None,
+                  "peak_source": f"{peak_src} hbm_gbs", "launches": n_merge,
+                  "avg_launch_ms": t_merge / max(1, n_merge)},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+                   "reasons": clk.get("reasons", []), "samples": clk.get("samples", 0)},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_sample_throughput(w, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": r["tflops"], "unit": "TFLOP/s", "cores": r["threads"], "kind": "oracle",
+            "sample": f"{r['rows']} query rows of {w.name} drawn uniformly over (batch, head, "
+                      f"row), full softmax row materialised in fp64; {r['seconds']:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, w, q_h, k_h, v_h, dev, out, ws, world) -> dict:
+    import torch
+
+    from online_softmax_exact_b200.schedules import ring_attention
+
+    qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    o_h = torch.empty(out[0].shape, dtype=torch.float32).pin_memory()
+    l_h = torch.empty(out[1].shape, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(qp, device=dev), torch.empty_like(kp, device=dev), \
+        torch.empty_like(vp, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = max(1, min(args.steps, 5))
+
+    def step():
+        qd.copy_(qp, non_blocking=True)
+        kd.copy_(kp, non_blocking=True)
+        vd.copy_(vp, non_blocking=True)
+        ring_attention(qd, kd, vd, n_chunks=w.n_chunks, causal=w.causal, scale=w.scale, out=out,
+                       workspace=ws, stream=stream)
+        o_h.copy_(out[0], non_blocking=True)
+        l_h.copy_(out[1], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    h2d = qp.numel() * 2 + kp.numel() * 2 + vp.numel() * 2
+    d2h = o_h.numel() * 4 + l_h.numel() * 4
+    return {"value": w.flops * steps * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="ring_32k")
+    ap.add_argument("--cpu-seconds", type=float, default=None,
+                    help="oracle CPU seconds (baseline sample; per step for --impl reference)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.cpu_seconds_set = args.cpu_seconds is not None
+    if args.cpu_seconds is None:
+        args.cpu_seconds = 12.0
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    from workloads import get
+
+    w = get(args.workload)
+    if w.schedule != "ring":
+        ap.error("the benchmark step is the ring schedule workload (ring_32k)")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

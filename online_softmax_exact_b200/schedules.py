@@ -64,13 +64,30 @@ def _alloc_out(q, n_chunks, out):
     return out
 
 
+class _NoTimer:
+    def __call__(self, kind: str):
+        return self
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_NO_TIMER = _NoTimer()
+
+
 def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None = None,
-                   out=None, workspace: Workspace | None = None, stream=None):
+                   out=None, workspace: Workspace | None = None, stream=None, timer=None):
     """Ring Attention's schedule on one GPU: query chunk i attends the key/value chunks
     of :func:`ring_order` one ring step at a time, then merges its partials.
 
+    ``timer(kind)``, if given, is entered around every launch ("partial" or "merge");
+    the benchmark uses it to bracket launches with CUDA events.
     Returns chunk-major (O [P,B,Hq,C,d], LSE [P,B,Hq,C]).
     """
+    timer = timer or _NO_TIMER
     B, Hq, N, d = q.shape
     bounds = chunk_bounds(N, n_chunks)
     C = N // n_chunks
@@ -84,28 +101,33 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
         if len(visit) == 1:
             # one part: the merge is the identity, so write the result in place
             ks, ke = bounds[visit[0]]
-            attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
-                             causal=causal, scale=scale, o=o_out[qi], lse=l_out[qi], stream=stream)
+            with timer("partial"):
+                attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks,
+                                 kv_len=ke - ks, causal=causal, scale=scale, o=o_out[qi],
+                                 lse=l_out[qi], stream=stream)
             continue
         for slot, kv in enumerate(visit):
             ks, ke = bounds[kv]
-            attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
-                             causal=causal, scale=scale, o=workspace.o[slot],
-                             lse=workspace.lse[slot], stream=stream)
+            with timer("partial"):
+                attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks,
+                                 kv_len=ke - ks, causal=causal, scale=scale,
+                                 o=workspace.o[slot], lse=workspace.lse[slot], stream=stream)
         n = len(visit)
-        attn_merge([workspace.o[i] for i in range(n)], [workspace.lse[i] for i in range(n)],
-                   o=o_out[qi], lse=l_out[qi], stream=stream)
+        with timer("merge"):
+            attn_merge([workspace.o[i] for i in range(n)], [workspace.lse[i] for i in range(n)],
+                       o=o_out[qi], lse=l_out[qi], stream=stream)
     return o_out, l_out
 
 
 def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], causal: bool,
                      scale: float | None = None, out=None, workspace: Workspace | None = None,
-                     stream=None):
+                     stream=None, timer=None):
     """ATTENTION2D's query x key/value grid on one GPU: every (query chunk, key/value
     chunk) cell is a partial attention (fragment-local statistics, section 3); each
     query chunk's partials are merged in the order ``merge_orders[i]`` (any order gives
     the same result, section 2). Returns chunk-major (O, LSE).
     """
+    timer = timer or _NO_TIMER
     B, Hq, N, d = q.shape
     bounds = chunk_bounds(N, n_chunks)
     C = N // n_chunks
@@ -120,11 +142,13 @@ def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], c
             raise ValueError("each merge order must be a permutation of the chunk indices")
         for kv in range(n_chunks):
             ks, ke = bounds[kv]
-            attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
-                             causal=causal, scale=scale, o=workspace.o[kv], lse=workspace.lse[kv],
-                             stream=stream)
-        attn_merge([workspace.o[i] for i in order], [workspace.lse[i] for i in order],
-                   o=o_out[qi], lse=l_out[qi], stream=stream)
+            with timer("partial"):
+                attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks,
+                                 kv_len=ke - ks, causal=causal, scale=scale, o=workspace.o[kv],
+                                 lse=workspace.lse[kv], stream=stream)
+        with timer("merge"):
+            attn_merge([workspace.o[i] for i in order], [workspace.lse[i] for i in order],
+                       o=o_out[qi], lse=l_out[qi], stream=stream)
     return o_out, l_out
 
 
