@@ -289,25 +289,28 @@ def run_reference(args, w) -> int:
 METRIC = "attention fwd TFLOP/s and % of bf16 tensor peak on 1 B200; merge HBM GB/s"
 
 
-def workload_config(w, world: int) -> dict:
+def workload_config(w, world: int, streams: int | None = None) -> dict:
     return {"workload": f"{w.name}: {w.description}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "N": w.N, "d": w.d, "causal": w.causal, "schedule": w.schedule,
             "n_chunks": w.n_chunks, "global_batch": w.B * world, "seq_len": w.N,
             "parallelism": "single GPU" if world == 1 else f"{world} independent replicas",
+            "streams": streams,
             "l2": "inputs larger than L2 (Q, K, V = 768 MiB per step); no flush"}
 
 
 class EventTimer:
-    """Brackets launches with CUDA events on the launching stream."""
+    """Brackets launches with CUDA events on the stream each launch is issued on."""
 
     def __init__(self, stream):
         self.stream = stream
         self.records = []  # (kind, start, end)
         self.enabled = False
         self._kind = None
+        self._stream = stream
 
-    def __call__(self, kind: str):
+    def __call__(self, kind: str, stream=None):
         self._kind = kind
+        self._stream = stream if stream is not None else self.stream
         return self
 
     def __enter__(self):
@@ -315,7 +318,7 @@ class EventTimer:
             import torch
 
             self._s = torch.cuda.Event(enable_timing=True)
-            self._s.record(self.stream)
+            self._s.record(self._stream)
         return self
 
     def __exit__(self, *exc):
@@ -323,15 +326,32 @@ class EventTimer:
             import torch
 
             e = torch.cuda.Event(enable_timing=True)
-            e.record(self.stream)
+            e.record(self._stream)
             self.records.append((self._kind, self._s, e))
         return False
 
-    def totals(self) -> dict:
-        out = {}
+    def totals(self, t0) -> dict:
+        """Per kind: (busy ms = union of its launch intervals, launches, summed ms).
+
+        With several streams, launches of one kind can overlap; the union counts the
+        device time during which at least one of them was in flight."""
+        spans = {}
         for kind, s, e in self.records:
-            t, n = out.get(kind, (0.0, 0))
-            out[kind] = (t + s.elapsed_time(e), n + 1)
+            spans.setdefault(kind, []).append((t0.elapsed_time(s), t0.elapsed_time(e)))
+        out = {}
+        for kind, iv in spans.items():
+            iv.sort()
+            busy, cur_a, cur_b = 0.0, None, None
+            for a, b in iv:
+                if cur_b is None or a > cur_b:
+                    if cur_b is not None:
+                        busy += cur_b - cur_a
+                    cur_a, cur_b = a, b
+                else:
+                    cur_b = max(cur_b, b)
+            if cur_b is not None:
+                busy += cur_b - cur_a
+            out[kind] = (busy, len(iv), sum(b - a for a, b in iv))
         return out
 
 
@@ -358,13 +378,13 @@ def run_ours(args, w) -> int:
     P, C = w.n_chunks, w.N // w.n_chunks
     out = (torch.empty((P, B, Hq, C, d), dtype=torch.float32, device=dev),
            torch.empty((P, B, Hq, C), dtype=torch.float32, device=dev))
-    ws = Workspace.for_shape(P, B, Hq, C, d, dev)
+    ws = Workspace.for_shape(P * args.streams, B, Hq, C, d, dev)
     stream = torch.cuda.current_stream(dev)
     timer = EventTimer(stream)
 
     def step():
         ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
-                       workspace=ws, stream=stream, timer=timer)
+                       workspace=ws, stream=stream, timer=timer, n_streams=args.streams)
 
     def barrier():
         if world > 1:
@@ -399,7 +419,7 @@ def run_ours(args, w) -> int:
     ms = t0.elapsed_time(t1)
     if osx.attn_device_status() != osx.ATTN_OK:
         raise RuntimeError("device-side wait ran out of time in the timed region")
-    tot = timer.totals()
+    tot = timer.totals(t0)
     clk = clocks.summary()
 
     ms_max = max_over_ranks(ms, dev)
@@ -410,14 +430,36 @@ def run_ours(args, w) -> int:
     fracs, merges = ring_step_plan(P, w.causal)
     full_pair_flops = 4.0 * B * Hq * C * C * d
     partial_flops_per_step = full_pair_flops * sum(fracs)
-    t_part, n_part = tot.get("partial", (0.0, 0))
-    t_merge, n_merge = tot.get("merge", (0.0, 0))
+    t_part, n_part, sum_part = tot.get("partial", (0.0, 0, 0.0))
     attn_achieved = partial_flops_per_step * args.steps / (t_part * 1e-3) / 1e12
     rows = B * Hq * C
-    mbytes = sum(merge_bytes(n, rows, d) for n in merges) * args.steps
-    merge_gbs = mbytes / (t_merge * 1e-3) / 1e9 if t_merge > 0 else None
     peak_t = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
     peak_h = peaks.get("hbm_gbs")
+
+    # ---- the merge kernel in isolation: the same step on one stream, so that merges do
+    # not share the device with attention launches of another stream
+    iso = EventTimer(stream)
+    n_iso = max(3, min(args.steps, 10))
+
+    def step1():
+        ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
+                       workspace=ws, stream=stream, timer=iso, n_streams=1)
+
+    step1()
+    torch.cuda.synchronize()
+    iso.enabled = True
+    t2 = torch.cuda.Event(enable_timing=True)
+    t2.record(stream)
+    for _ in range(n_iso):
+        step1()
+    torch.cuda.synchronize()
+    iso.enabled = False
+    tot1 = iso.totals(t2)
+    t_merge, n_merge, sum_merge = tot1.get("merge", (0.0, 0, 0.0))
+    t_part1, _, _ = tot1.get("partial", (0.0, 0, 0.0))
+    mbytes = sum(merge_bytes(n, rows, d) for n in merges) * n_iso
+    merge_gbs = mbytes / (t_merge * 1e-3) / 1e9 if t_merge > 0 else None
+    attn_single = partial_flops_per_step * n_iso / (t_part1 * 1e-3) / 1e12 if t_part1 else None
 
     # ---- end to end through the public API with pinned host buffers
     e2e = run_e2e(args, w, q_h, k_h, v_h, dev, out, ws, world)
@@ -429,7 +471,7 @@ def run_ours(args, w) -> int:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: bf16 N(0,1) from a seeded torch CPU generator",
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, args.streams),
         "pct_of_bf16_peak": 100.0 * (value / world) / peak_t,
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128> (attn_fwd_partial)",
                      "achieved": attn_achieved, "peak": peak_t, "unit": "TFLOP/s",
@@ -437,12 +479,19 @@ def run_ours(args, w) -> int:
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a "
                                     f"long back-to-back loop)",
                      "traffic": None,
-                     "launches": n_part, "avg_launch_ms": t_part / max(1, n_part)},
+                     "launches": n_part, "busy_ms": t_part, "summed_launch_ms": sum_part,
+                     "timing": "achieved = algorithmic FLOPs of all attention launches in the "
+                               "timed region / the device time during which at least one was "
+                               "in flight (union of CUDA-event intervals on the launching "
+                               "streams)",
+                     "achieved_single_stream": attn_single},
         "merge": {"bound": "hbm", "kernel": "attn_merge_kernel<128>", "achieved": merge_gbs,
                   "peak": peak_h, "unit": "GB/s",
                   "frac": (merge_gbs / peak_h) if merge_gbs else None,
                   "peak_source": f"{peak_src} hbm_gbs", "launches": n_merge,
-                  "avg_launch_ms": t_merge / max(1, n_merge)},
+                  "busy_ms": t_merge, "summed_launch_ms": sum_merge,
+                  "timing": f"the same ring step on one stream, {n_iso} steps after the timed "
+                            "region; algorithmic bytes / CUDA-event time of the merge launches"},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
@@ -480,7 +529,7 @@ def run_e2e(args, w, q_h, k_h, v_h, dev, out, ws, world) -> dict:
         kd.copy_(kp, non_blocking=True)
         vd.copy_(vp, non_blocking=True)
         ring_attention(qd, kd, vd, n_chunks=w.n_chunks, causal=w.causal, scale=w.scale, out=out,
-                       workspace=ws, stream=stream)
+                       workspace=ws, stream=stream, n_streams=args.streams)
         o_h.copy_(out[0], non_blocking=True)
         l_h.copy_(out[1], non_blocking=True)
 
@@ -508,6 +557,8 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="ring_32k")
+    ap.add_argument("--streams", type=int, default=2,
+                    help="CUDA streams the ring schedule spreads its query chunks over")
     ap.add_argument("--cpu-seconds", type=float, default=None,
                     help="oracle CPU seconds (baseline sample; per step for --impl reference)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

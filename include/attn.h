@@ -121,10 +121,11 @@ attn_status_t attn_fwd_partial(const void* q, const void* k_chunk, const void* v
  * fp32 rounding.
  *
  *   o_parts, lse_parts  HOST arrays of n_parts DEVICE pointers: fp32 [rows][d]
- *                       (16-byte aligned) and fp32 [rows] (4-byte aligned)
+ *                       (32-byte aligned: rows move as 256-bit loads) and fp32
+ *                       [rows] (4-byte aligned)
  *   n_parts             1 .. ATTN_MAX_MERGE_PARTS
- *   o, lse              device, fp32 [rows][d] and [rows] (written); must not
- *                       overlap any part
+ *   o, lse              device, fp32 [rows][d] (32-byte aligned) and [rows]
+ *                       (written); must not overlap any part
  *   rows >= 1; d in {64, 128}
  */
 attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_parts,

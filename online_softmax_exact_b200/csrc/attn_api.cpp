@@ -125,7 +125,7 @@ attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_pa
                          float* o, float* lse, int64_t rows, int d, void* stream) {
   if (!o_parts || !lse_parts || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (n_parts < 1 || rows < 1) return ATTN_ERR_INVALID_ARG;
-  if (!aligned(o, 16) || !aligned(lse, 4)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(o, 32) || !aligned(lse, 4)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (n_parts > ATTN_MAX_MERGE_PARTS) return ATTN_ERR_UNSUPPORTED;
   if (rows > (int64_t(1) << 40)) return ATTN_ERR_UNSUPPORTED;
@@ -134,7 +134,7 @@ attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_pa
   if (overlap(so, sl)) return ATTN_ERR_INVALID_ARG;
   for (int i = 0; i < n_parts; ++i) {
     if (!o_parts[i] || !lse_parts[i]) return ATTN_ERR_INVALID_ARG;
-    if (!aligned(o_parts[i], 16) || !aligned(lse_parts[i], 4)) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(o_parts[i], 32) || !aligned(lse_parts[i], 4)) return ATTN_ERR_INVALID_ARG;
     const Span po = span(o_parts[i], (uint64_t)rows * d * 4);
     const Span pl = span(lse_parts[i], (uint64_t)rows * 4);
     if (overlap(so, po) || overlap(so, pl) || overlap(sl, po) || overlap(sl, pl))

@@ -48,6 +48,7 @@ struct FwdParams {
   int n_qpairs;        // ceil(Nq / 256)
   int n_units;         // n_qpairs * BH
   int n_kv_tiles;      // ceil(Nkv / 128)
+  int o_vec8;          // O is 32-byte aligned: store rows with 256-bit stores
 };
 
 template <int D>
@@ -65,7 +66,13 @@ struct FwdCfg {
   static constexpr int kNumBars = 2 + 4 * kStages + 6 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
-  static constexpr int kThreads = 320;
+  // warpgroups: 0 and 1 softmax (Q tiles 0 and 1), 2 = {TMA producer, MMA issuer, 2 idle}
+  static constexpr int kThreads = 384;
+  // registers per thread: 168 at launch for all (each SM sub-partition hosts one warp
+  // of each warpgroup); after setmaxnreg the softmax warpgroups hold 216 and warpgroup 2
+  // holds 72 (216 + 216 + 72 = 3 * 168, the launch's total)
+  static constexpr int kRegsSoftmax = 216;
+  static constexpr int kRegsOther = 72;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 };
 
@@ -86,8 +93,53 @@ __device__ __forceinline__ int unit_kv_tiles(const FwdParams& p, int qp) {
   return n < p.n_kv_tiles ? (int)n : p.n_kv_tiles;
 }
 
+// One row's P for one 128-key tile: x = S * scale*log2(e) - m (packed pairs), P = 2^x,
+// written back to TMEM as bf16 pairs over the first 64 columns of S; returns sum(P).
+// Masked tiles send every element through ex2 (so that -inf gives exactly 0); other
+// tiles send 4 of every 16 pairs through the FMA-pipe polynomial to share the load with
+// the exp unit.
+template <bool kMasked>
+__device__ __forceinline__ float softmax_tile(uint32_t (&s)[4][32], uint32_t tS, float c,
+                                              float m_use, int climit) {
+  const uint64_t C2 = f2_pack(c, c);
+  const uint64_t NM2 = f2_pack(-m_use, -m_use);
+  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint64_t X = f2_fma(f2_pack(__uint_as_float(s[q4][2 * i]),
+                                        __uint_as_float(s[q4][2 * i + 1])), C2, NM2);
+      float x0, x1, e0, e1;
+      f2_unpack(X, x0, x1);
+      if (kMasked) {
+        if (q4 * 32 + 2 * i > climit) x0 = -INFINITY;
+        if (q4 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
+        e0 = ex2_approx(x0);
+        e1 = ex2_approx(x1);
+      } else if (i >= 12) {
+        exp2_poly_pair(x0, x1, e0, e1);
+      } else {
+        e0 = ex2_approx(x0);
+        e1 = ex2_approx(x1);
+      }
+      if (i & 1)
+        acc1 = f2_add(acc1, f2_pack(e0, e1));
+      else
+        acc0 = f2_add(acc0, f2_pack(e0, e1));
+      pk[i] = pack_bf16x2(e0, e1);
+    }
+    tmem_st16(tS + q4 * 16, pk);
+  }
+  float a, b, cc, d;
+  f2_unpack(acc0, a, b);
+  f2_unpack(acc1, cc, d);
+  return (a + b) + (cc + d);
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D>;
@@ -119,7 +171,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(B_SF + t), 1);
-      mbar_init(bar(B_PF + t), 128);
+      mbar_init(bar(B_PF + t), 4);  // one arrival per softmax warp
       mbar_init(bar(B_OD + t), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
@@ -140,6 +192,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   const int G = gridDim.x;
 
+  if (warp >= 8) {
+  regs_decrease<C::kRegsOther>();
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -253,7 +307,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (++vs == C::kStages) { vs = 0; vph ^= 1; }
       }
     }
+  }
   } else {
+    regs_increase<C::kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax warpgroups
     const int t = warp / 4;                 // which Q tile of the unit
     const int wq = warp % 4;                // warp's TMEM lane quarter
@@ -318,7 +374,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         long long cl = lim_row - kbase;
         const int climit = cl < -1 ? -1 : (cl > 127 ? 127 : (int)cl);
 
-        float mx = -INFINITY;
         if (need_mask) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
@@ -326,16 +381,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int i = 0; i < 32; ++i)
               if (q4 * 32 + i > climit) s[q4][i] = __float_as_uint(-INFINITY);
         }
+        float mx;
         {
           float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            m0 = fmaxf(m0, __uint_as_float(s[0][i]));
-            m1 = fmaxf(m1, __uint_as_float(s[1][i]));
-            m2 = fmaxf(m2, __uint_as_float(s[2][i]));
-            m3 = fmaxf(m3, __uint_as_float(s[3][i]));
+          for (int i = 0; i < 16; ++i) {
+            m0 = fmax3(m0, __uint_as_float(s[0][2 * i]), __uint_as_float(s[0][2 * i + 1]));
+            m1 = fmax3(m1, __uint_as_float(s[1][2 * i]), __uint_as_float(s[1][2 * i + 1]));
+            m2 = fmax3(m2, __uint_as_float(s[2][2 * i]), __uint_as_float(s[2][2 * i + 1]));
+            m3 = fmax3(m3, __uint_as_float(s[3][2 * i]), __uint_as_float(s[3][2 * i + 1]));
           }
-          mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+          mx = fmax3(m0, m1, fmaxf(m2, m3));
         }
         const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * c;
         const float m_new = (m_tile > m + 8.0f) ? m_tile : m;
@@ -343,27 +399,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
 
-        float sum = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0 = fmaf(__uint_as_float(s[q4][2 * i]), c, -m_use);
-            float x1 = fmaf(__uint_as_float(s[q4][2 * i + 1]), c, -m_use);
-            if (need_mask) {
-              if (q4 * 32 + 2 * i > climit) x0 = -INFINITY;
-              if (q4 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
-            }
-            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-            s0 += e0;
-            s1 += e1;
-            pk[i] = pack_bf16x2(e0, e1);
-          }
-          sum += s0 + s1;
-          tmem_st16(tS + q4 * 16, pk);
-        }
+        float sum = need_mask ? softmax_tile<true>(s, tS, c, m_use, climit)
+                              : softmax_tile<false>(s, tS, c, m_use, climit);
         l = l * alpha + sum;
 
         // rescale this warp's rows of O when any of them moved its maximum
@@ -383,7 +420,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m = m_new;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(B_PF + t));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PF + t));
       }
       if (!ok) break;
 
@@ -401,12 +439,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld32(tO + q4 * 32, ov);
         tmem_ld_wait(ov);
         if (row_valid) {
-          float4* o4 = reinterpret_cast<float4*>(orow + q4 * 32);
+          float* dst = orow + q4 * 32;
+          if (p.o_vec8) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o4[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
-                                __uint_as_float(ov[4 * i + 2]) * inv_l,
-                                __uint_as_float(ov[4 * i + 3]) * inv_l);
+            for (int i = 0; i < 4; ++i)
+              st_global_v8(dst + 8 * i, __uint_as_float(ov[8 * i]) * inv_l,
+                           __uint_as_float(ov[8 * i + 1]) * inv_l,
+                           __uint_as_float(ov[8 * i + 2]) * inv_l,
+                           __uint_as_float(ov[8 * i + 3]) * inv_l,
+                           __uint_as_float(ov[8 * i + 4]) * inv_l,
+                           __uint_as_float(ov[8 * i + 5]) * inv_l,
+                           __uint_as_float(ov[8 * i + 6]) * inv_l,
+                           __uint_as_float(ov[8 * i + 7]) * inv_l);
+          } else {
+            float4* o4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              o4[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l,
+                                  __uint_as_float(ov[4 * i + 1]) * inv_l,
+                                  __uint_as_float(ov[4 * i + 2]) * inv_l,
+                                  __uint_as_float(ov[4 * i + 3]) * inv_l);
+          }
         }
       }
       if (row_valid) {

@@ -85,6 +85,7 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   p.n_units = static_cast<int>(units);
   p.n_kv_tiles = static_cast<int>((a.Nkv + 127) / 128);
+  p.o_vec8 = (reinterpret_cast<uintptr_t>(a.o) % 32) == 0 ? 1 : 0;
   const int grid = p.n_units < di.num_sms ? p.n_units : di.num_sms;
   attn_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -92,16 +93,23 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
   return ATTN_OK;
 }
 
-template <int D>
-int launch_merge_d(const MergeParams& p, const DeviceInfo& di, cudaStream_t stream) {
-  constexpr int rpb = 256 / (D / 4);
-  long long blocks = (p.rows + rpb - 1) / rpb;
-  const long long cap = (long long)di.num_sms * 8;
+template <int D, int G>
+int launch_merge_dg(const MergeParams& p, const DeviceInfo& di, cudaStream_t stream) {
+  constexpr int rows_per_block = (256 / (D / 8)) * (8 / G);
+  long long blocks = (p.rows + rows_per_block - 1) / rows_per_block;
+  const long long cap = (long long)di.num_sms * 4;
   if (blocks > cap) blocks = cap;
-  attn_merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(p);
+  attn_merge_kernel<D, G><<<(unsigned)blocks, 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return ATTN_OK;
+}
+
+template <int D>
+int launch_merge_d(const MergeParams& p, const DeviceInfo& di, cudaStream_t stream) {
+  if (p.n <= 2) return launch_merge_dg<D, 2>(p, di, stream);
+  if (p.n <= 4) return launch_merge_dg<D, 4>(p, di, stream);
+  return launch_merge_dg<D, 8>(p, di, stream);
 }
 
 }  // namespace

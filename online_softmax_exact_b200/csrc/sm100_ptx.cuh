@@ -1,6 +1,6 @@
 // sm100_ptx.cuh - thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers with bounded waits, TMA tiled loads, and the tcgen05 tensor-core / tensor
-// memory (TMEM) instructions. Only instructions are wrapped here; no arithmetic.
+// mbarriers with bounded waits, TMA tiled loads, the tcgen05 tensor-core / tensor
+// memory (TMEM) instructions, packed fp32 pairs, and a polynomial 2^x on the FMA pipe.
 #pragma once
 
 #include <cstdint>
@@ -110,6 +110,16 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
+}
+
+// Register reallocation between warpgroups (all 128 threads of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -256,6 +266,77 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
+}
+
+// Coefficients of p(f) ~ 2^f on [-1/2, 1/2], p(f) = 1 + c1 f + c2 f^2 + c3 f^3, fitted by
+// exp2_poly_fit.py (max relative error 1.03e-4 evaluated in fp32).
+constexpr float kExp2C1 = 6.932863593e-01f;
+constexpr float kExp2C2 = 2.422038764e-01f;
+constexpr float kExp2C3 = 5.498712510e-02f;
+
+// 256-bit global store of 8 floats (address 32-byte aligned)
+__device__ __forceinline__ void st_global_v8(float* p, float a0, float a1, float a2, float a3,
+                                             float a4, float a5, float a6, float a7) {
+  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(a0), "f"(a1),
+               "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7)
+               : "memory");
+}
+
+// three-input maximum (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// packed fp32 pairs (sm_100): {lo, hi} in one 64-bit register pair
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of finite x <= 64 on the FMA pipe: x clamped below at -125, n =
+// round(x) by the 1.5*2^23 shifter, f = x - n in [-1/2, 1/2], 2^f by a degree-3
+// polynomial (coefficients fitted by exp2_poly_fit.py for minimum relative error:
+// 1.03e-4 at most), and n added to the exponent field. Inputs below -125 give 2^-125
+// or so instead of a smaller value; callers only pass rows whose denominator is >= 1.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  const uint64_t X = f2_pack(x0, x1);
+  const uint64_t SH = f2_pack(kShift, kShift);
+  const uint64_t J = f2_add(X, SH);       // kShift + round(x): n in the low mantissa bits
+  const uint64_t R = f2_sub(J, SH);       // round(x) as a float
+  const uint64_t F = f2_sub(X, R);        // f in [-1/2, 1/2]
+  uint64_t P = f2_fma(f2_pack(kExp2C3, kExp2C3), F, f2_pack(kExp2C2, kExp2C2));
+  P = f2_fma(P, F, f2_pack(kExp2C1, kExp2C1));
+  P = f2_fma(P, F, f2_pack(1.0f, 1.0f));
+  float p0, p1, j0, j1;
+  f2_unpack(P, p0, p1);
+  f2_unpack(J, j0, j1);
+  // (kShift + n) << 23 leaves exactly n << 23 in 32 bits
+  y0 = __uint_as_float(__float_as_uint(j0) * 8388608u + __float_as_uint(p0));
+  y1 = __uint_as_float(__float_as_uint(j1) * 8388608u + __float_as_uint(p1));
 }
 
 }  // namespace osx

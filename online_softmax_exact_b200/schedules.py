@@ -65,7 +65,7 @@ def _alloc_out(q, n_chunks, out):
 
 
 class _NoTimer:
-    def __call__(self, kind: str):
+    def __call__(self, kind: str, stream=None):
         return self
 
     def __enter__(self):
@@ -78,13 +78,51 @@ class _NoTimer:
 _NO_TIMER = _NoTimer()
 
 
+def balance_streams(costs: list[float], n_streams: int) -> list[int]:
+    """Assign query chunks to streams, heaviest first onto the least-loaded stream."""
+    load = [0.0] * n_streams
+    assign = [0] * len(costs)
+    for i in sorted(range(len(costs)), key=lambda i: -costs[i]):
+        s = min(range(n_streams), key=lambda j: load[j])
+        assign[i] = s
+        load[s] += costs[i]
+    return assign
+
+
+class _Streams:
+    """Fork work from ``main`` onto side streams and join it back."""
+
+    def __init__(self, main, n: int, device):
+        self.main = main
+        self.side = [main] if n <= 1 else [torch.cuda.Stream(device) for _ in range(n)]
+        if n > 1:
+            ev = torch.cuda.Event()
+            ev.record(main)
+            for s in self.side:
+                s.wait_event(ev)
+
+    def join(self, tensors):
+        if len(self.side) == 1:
+            return
+        for s in self.side:
+            ev = torch.cuda.Event()
+            ev.record(s)
+            self.main.wait_event(ev)
+            for t in tensors:
+                t.record_stream(s)
+
+
 def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None = None,
-                   out=None, workspace: Workspace | None = None, stream=None, timer=None):
+                   out=None, workspace: Workspace | None = None, stream=None, timer=None,
+                   n_streams: int = 1):
     """Ring Attention's schedule on one GPU: query chunk i attends the key/value chunks
     of :func:`ring_order` one ring step at a time, then merges its partials.
 
-    ``timer(kind)``, if given, is entered around every launch ("partial" or "merge");
-    the benchmark uses it to bracket launches with CUDA events.
+    With ``n_streams`` > 1 the query chunks are spread over that many CUDA streams
+    (balanced by their number of partials), so that one launch's tail overlaps the next
+    launch; each chunk's partials and merge stay in order on its stream, and the result
+    is joined back into ``stream``. ``timer(kind)``, if given, is entered around every
+    launch ("partial" or "merge") with the launching stream as argument.
     Returns chunk-major (O [P,B,Hq,C,d], LSE [P,B,Hq,C]).
     """
     timer = timer or _NO_TIMER
@@ -94,34 +132,45 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
     order = ring_order(n_chunks, causal)
     o_out, l_out = _alloc_out(q, n_chunks, out)
     slots = max(len(x) for x in order)
-    if workspace is None or workspace.o.shape[0] < slots or workspace.o.shape[1:] != (B, Hq, C, d):
-        workspace = Workspace.for_shape(slots, B, Hq, C, d, q.device)
-    for qi, visit in enumerate(order):
+    n_streams = max(1, min(n_streams, n_chunks))
+    need = slots * n_streams
+    if workspace is None or workspace.o.shape[0] < need or workspace.o.shape[1:] != (B, Hq, C, d):
+        workspace = Workspace.for_shape(need, B, Hq, C, d, q.device)
+    main = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = _Streams(main, n_streams, q.device)
+    assign = balance_streams([float(len(x)) for x in order], n_streams)
+    for qi in sorted(range(n_chunks), key=lambda i: -len(order[i])):
+        visit = order[qi]
+        s_idx = assign[qi]
+        s = st.side[s_idx]
+        base = s_idx * slots
         qs, qe = bounds[qi]
         if len(visit) == 1:
             # one part: the merge is the identity, so write the result in place
             ks, ke = bounds[visit[0]]
-            with timer("partial"):
+            with timer("partial", s):
                 attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks,
                                  kv_len=ke - ks, causal=causal, scale=scale, o=o_out[qi],
-                                 lse=l_out[qi], stream=stream)
+                                 lse=l_out[qi], stream=s)
             continue
-        for slot, kv in enumerate(visit):
+        for j, kv in enumerate(visit):
             ks, ke = bounds[kv]
-            with timer("partial"):
+            with timer("partial", s):
                 attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks,
                                  kv_len=ke - ks, causal=causal, scale=scale,
-                                 o=workspace.o[slot], lse=workspace.lse[slot], stream=stream)
+                                 o=workspace.o[base + j], lse=workspace.lse[base + j], stream=s)
         n = len(visit)
-        with timer("merge"):
-            attn_merge([workspace.o[i] for i in range(n)], [workspace.lse[i] for i in range(n)],
-                       o=o_out[qi], lse=l_out[qi], stream=stream)
+        with timer("merge", s):
+            attn_merge([workspace.o[base + i] for i in range(n)],
+                       [workspace.lse[base + i] for i in range(n)],
+                       o=o_out[qi], lse=l_out[qi], stream=s)
+    st.join([q, k, v, o_out, l_out, workspace.o, workspace.lse])
     return o_out, l_out
 
 
 def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], causal: bool,
                      scale: float | None = None, out=None, workspace: Workspace | None = None,
-                     stream=None, timer=None):
+                     stream=None, timer=None, n_streams: int = 1):
     """ATTENTION2D's query x key/value grid on one GPU: every (query chunk, key/value
     chunk) cell is a partial attention (fragment-local statistics, section 3); each
     query chunk's partials are merged in the order ``merge_orders[i]`` (any order gives
@@ -132,23 +181,32 @@ def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], c
     bounds = chunk_bounds(N, n_chunks)
     C = N // n_chunks
     o_out, l_out = _alloc_out(q, n_chunks, out)
-    if workspace is None or workspace.o.shape[0] < n_chunks or \
+    n_streams = max(1, min(n_streams, n_chunks))
+    need = n_chunks * n_streams
+    if workspace is None or workspace.o.shape[0] < need or \
             workspace.o.shape[1:] != (B, Hq, C, d):
-        workspace = Workspace.for_shape(n_chunks, B, Hq, C, d, q.device)
+        workspace = Workspace.for_shape(need, B, Hq, C, d, q.device)
+    main = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = _Streams(main, n_streams, q.device)
     for qi in range(n_chunks):
+        s = st.side[qi % n_streams]
+        base = (qi % n_streams) * n_chunks
         qs, qe = bounds[qi]
         order = merge_orders[qi]
         if sorted(order) != list(range(n_chunks)):
             raise ValueError("each merge order must be a permutation of the chunk indices")
         for kv in range(n_chunks):
             ks, ke = bounds[kv]
-            with timer("partial"):
+            with timer("partial", s):
                 attn_fwd_partial(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks,
-                                 kv_len=ke - ks, causal=causal, scale=scale, o=workspace.o[kv],
-                                 lse=workspace.lse[kv], stream=stream)
-        with timer("merge"):
-            attn_merge([workspace.o[i] for i in order], [workspace.lse[i] for i in order],
-                       o=o_out[qi], lse=l_out[qi], stream=stream)
+                                 kv_len=ke - ks, causal=causal, scale=scale,
+                                 o=workspace.o[base + kv], lse=workspace.lse[base + kv],
+                                 stream=s)
+        with timer("merge", s):
+            attn_merge([workspace.o[base + i] for i in order],
+                       [workspace.lse[base + i] for i in order],
+                       o=o_out[qi], lse=l_out[qi], stream=s)
+    st.join([q, k, v, o_out, l_out, workspace.o, workspace.lse])
     return o_out, l_out
 
 

@@ -118,6 +118,8 @@ def test_merge_argument_checks(lib):
     assert merge(n=65, parts_o=[A] * 65, parts_l=[4 * A] * 65) == ATTN_ERR_UNSUPPORTED
     assert merge(parts_o=[A, None]) == ATTN_ERR_INVALID_ARG
     assert merge(parts_o=[A + 4, 2 * A]) == ATTN_ERR_INVALID_ARG  # misaligned part
+    assert merge(parts_o=[A + 16, 2 * A]) == ATTN_ERR_INVALID_ARG  # parts need 32 bytes
+    assert merge(o=16 * A + 16) == ATTN_ERR_INVALID_ARG           # so does the output
     assert merge(o=A) == ATTN_ERR_INVALID_ARG                     # output aliases a part
     assert merge(lse=4 * A) == ATTN_ERR_INVALID_ARG               # lse aliases a part
 

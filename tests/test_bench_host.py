@@ -116,3 +116,19 @@ def test_reference_arm_other_ranks_do_nothing():
                         "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
                        env=env, timeout=120, cwd=ROOT)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_event_timer_busy_time_is_the_union_of_intervals():
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    t = bench.EventTimer(None)
+    t.records = [("partial", Ev(0), Ev(2)), ("partial", Ev(1), Ev(3)),
+                 ("partial", Ev(5), Ev(6)), ("merge", Ev(3), Ev(4))]
+    tot = t.totals(Ev(0))
+    assert tot["partial"] == (4.0, 3, 5.0)      # [0,3] and [5,6]
+    assert tot["merge"] == (1.0, 1, 1.0)
