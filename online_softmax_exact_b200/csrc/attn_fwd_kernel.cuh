@@ -9,23 +9,29 @@
 //
 // B200 mapping (our design, not the page's):
 //   * one CTA per SM (persistent), work unit = 256 query rows of one (batch, head),
-//     held as two 128-row tiles that two softmax warpgroups process in ping-pong, so
-//     the tensor core works on one tile while the other tile's softmax runs;
-//   * warp 8 issues TMA loads (Q tiles once per unit, K and V tiles through a ring of
+//     held as two 128-row tiles in ping-pong: the tensor core works on one tile while
+//     the other tile's softmax runs;
+//   * warp 16 issues TMA loads (Q tiles once per unit, K and V tiles through a ring of
 //     shared-memory stages, 128-byte swizzle);
-//   * warp 9 owns tensor memory and issues tcgen05.mma from one thread:
+//   * warp 17 owns tensor memory and issues tcgen05.mma from one thread:
 //     S_t = Q_t K_j^T (both operands in shared memory) into TMEM, then O_t += P_t V_j
 //     with P_t read from TMEM (written there by the softmax warps over S_t's columns);
-//   * softmax warpgroup t: thread r owns query row r of tile t (TMEM lane r), reads its
-//     128 scores with tcgen05.ld, masks, takes the row maximum, exponentiates with
-//     ex2, sums, packs P to bf16 and writes it back with tcgen05.st. The maximum used
-//     for the exponent is only moved when the tile maximum exceeds it by more than
-//     2^8 (exactness is kept because the same stale maximum is used for numerator and
-//     denominator); when it moves, the warp rescales its rows of O in TMEM;
+//   * four softmax warpgroups: warpgroup 2t + h handles key half h (64 of the 128 keys of
+//     a tile) of every row of tile t, one row per thread (TMEM lane = row), so each
+//     row's softmax is split over two threads that exchange their half-row maxima (and
+//     at the end their half denominators) through shared memory under a 64-thread
+//     named barrier. A thread reads its 64 scores with tcgen05.ld, exponentiates with
+//     ex2, sums, packs P to bf16 and writes it back with tcgen05.st. The exponent base
+//     is the running maximum m, moved only when a tile maximum exceeds it by more than
+//     8 (log2 units); exactness is kept because numerator and denominator share the
+//     same base. In the common case the exponentials are computed against the current
+//     m while the tile maximum is reduced alongside, and redone only if m moves; when
+//     m moves the threads rescale their halves of O in TMEM;
 //   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32.
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [384,384+D). P_t (bf16 pairs) overwrites S_t columns [0,64) after S_t is read.
+// O_1 [384,384+D). Half h of P_t (bf16 pairs) overwrites S_t columns [64h, 64h+32),
+// inside that half's own score columns.
 //
 // All mbarrier waits are bounded (see mbar_wait); on time-out the kernel records it in
 // the device status word, lets in-flight work drain, frees TMEM and returns.
@@ -65,15 +71,22 @@ struct FwdCfg {
   // s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 2 + 4 * kStages + 6 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
-  // warpgroups: 0 and 1 softmax (Q tiles 0 and 1), 2 = {TMA producer, MMA issuer, 2 idle}
-  static constexpr int kThreads = 384;
-  // registers per thread: 168 at launch for all (each SM sub-partition hosts one warp
-  // of each warpgroup); after setmaxnreg the softmax warpgroups hold 216 and warpgroup 2
-  // holds 72 (216 + 216 + 72 = 3 * 168, the launch's total)
-  static constexpr int kRegsSoftmax = 216;
-  static constexpr int kRegsOther = 72;
+  // half-row exchange: maxima [tile][parity][half][row], denominators [tile][half][row]
+  static constexpr uint32_t kXchOff = (kMiscOff + 16 + 127) & ~127u;
+  static constexpr uint32_t kXlOff = kXchOff + 2 * 2 * 2 * 128 * 4;
+  static constexpr uint32_t kSmemBytes = kXlOff + 2 * 2 * 128 * 4 + 1024;  // + alignment slack
+  // warpgroups 0-3: softmax (tile t = wg / 2, key half h = wg % 2);
+  // warpgroup 4: {TMA producer, MMA issuer, 2 idle}
+  static constexpr int kThreads = 640;
+  static constexpr int kWarpProducer = 16, kWarpMma = 17;
+  // Registers per thread: 96 at launch for all (each SM sub-partition hosts one warp of
+  // each warpgroup); after setmaxnreg the softmax warpgroups hold 104 and warpgroup 4
+  // holds 64 (4 * 104 + 64 = 5 * 96, the launch's total).
+  static constexpr int kRegsSoftmax = 104;
+  static constexpr int kRegsOther = 64;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+  // In each 16-pair chunk of a half row, pairs i >= kPolyFrom use the FMA-pipe 2^x.
+  static constexpr int kPolyFrom = 16;
 };
 
 __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
@@ -93,53 +106,59 @@ __device__ __forceinline__ int unit_kv_tiles(const FwdParams& p, int qp) {
   return n < p.n_kv_tiles ? (int)n : p.n_kv_tiles;
 }
 
-// One row's P for one 128-key tile: x = S * scale*log2(e) - m (packed pairs), P = 2^x,
-// written back to TMEM as bf16 pairs over the first 64 columns of S; returns sum(P).
-// Masked tiles send every element through ex2 (so that -inf gives exactly 0); other
-// tiles send 4 of every 16 pairs through the FMA-pipe polynomial to share the load with
-// the exp unit.
-template <bool kMasked>
-__device__ __forceinline__ float softmax_tile(uint32_t (&s)[4][32], uint32_t tS, float c,
-                                              float m_use, int climit) {
+// One thread's half row of P for one 128-key tile (64 scores in s): x = S * c - m
+// (packed pairs), P = 2^x, written to TMEM as 32 columns of bf16 pairs at tP; returns
+// sum(P). Masked tiles send every element through ex2 (so that -inf gives exactly 0).
+// With kWithMax it also reduces the half-row maximum of the raw scores alongside.
+template <bool kMasked, bool kWithMax, int kPolyFrom>
+__device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP, float c,
+                                              float m_use, int climit, float* tile_max) {
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   const uint64_t C2 = f2_pack(c, c);
   const uint64_t NM2 = f2_pack(-m_use, -m_use);
-  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
+  for (int q2 = 0; q2 < 2; ++q2) {
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint64_t X = f2_fma(f2_pack(__uint_as_float(s[q4][2 * i]),
-                                        __uint_as_float(s[q4][2 * i + 1])), C2, NM2);
+      const float s0 = __uint_as_float(s[q2][2 * i]), s1 = __uint_as_float(s[q2][2 * i + 1]);
+      if (kWithMax) {
+        if (i & 1)
+          mx1 = fmax3(mx1, s0, s1);
+        else
+          mx0 = fmax3(mx0, s0, s1);
+      }
       float x0, x1, e0, e1;
-      f2_unpack(X, x0, x1);
+      f2_unpack(f2_fma(f2_pack(s0, s1), C2, NM2), x0, x1);
       if (kMasked) {
-        if (q4 * 32 + 2 * i > climit) x0 = -INFINITY;
-        if (q4 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
+        if (q2 * 32 + 2 * i > climit) x0 = -INFINITY;
+        if (q2 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
         e0 = ex2_approx(x0);
         e1 = ex2_approx(x1);
-      } else if (i >= 12) {
+      } else if (i >= kPolyFrom) {
         exp2_poly_pair(x0, x1, e0, e1);
       } else {
         e0 = ex2_approx(x0);
         e1 = ex2_approx(x1);
       }
-      if (i & 1)
-        acc1 = f2_add(acc1, f2_pack(e0, e1));
-      else
-        acc0 = f2_add(acc0, f2_pack(e0, e1));
+      if (i & 1) {
+        a2 += e0;
+        a3 += e1;
+      } else {
+        a0 += e0;
+        a1 += e1;
+      }
       pk[i] = pack_bf16x2(e0, e1);
     }
-    tmem_st16(tS + q4 * 16, pk);
+    tmem_st16(tP + q2 * 16, pk);
   }
-  float a, b, cc, d;
-  f2_unpack(acc0, a, b);
-  f2_unpack(acc1, cc, d);
-  return (a + b) + (cc + d);
+  if (kWithMax) *tile_max = fmaxf(mx0, mx1);
+  return (a0 + a1) + (a2 + a3);
 }
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D>;
@@ -150,6 +169,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  float* xch = reinterpret_cast<float*>(smem + C::kXchOff);
+  float* xl = reinterpret_cast<float*>(smem + C::kXlOff);
 
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int B_QF = 0, B_QE = 1;
@@ -171,17 +192,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(B_SF + t), 1);
-      mbar_init(bar(B_PF + t), 4);  // one arrival per softmax warp
+      mbar_init(bar(B_PF + t), 8);  // one arrival per softmax warp of the tile
       mbar_init(bar(B_OD + t), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == C::kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == C::kWarpProducer && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -192,134 +213,160 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   const int G = gridDim.x;
 
-  if (warp >= 8) {
-  regs_decrease<C::kRegsOther>();
-  if (warp == 8) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int u = unit_for_round(r, blockIdx.x, G);
-        if (u >= p.n_units) break;
-        const int qp = p.n_qpairs - 1 - u / p.BH;
-        const int bh = u % p.BH;
-        const int n = unit_kv_tiles(p, qp);
-        if (n == 0) continue;
-        const int kvh = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
-        if (!(ok = mbar_wait(bar(B_QE), (qcount & 1) ^ 1, abort_flag, p.status))) break;
-        ++qcount;
-        mbar_arrive_expect_tx(bar(B_QF), 2 * C::kTileBytes);
-        for (int t = 0; t < 2; ++t)
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + h * 16384, &tmQ, bar(B_QF), h * 64,
-                        qp * 256 + t * 128, bh);
-        for (int j = 0; j < n; ++j) {
-          if (!(ok = mbar_wait(bar(B_KE + ks), kph ^ 1, abort_flag, p.status))) break;
-          mbar_arrive_expect_tx(bar(B_KF + ks), C::kTileBytes);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sbase + C::kKOff + ks * C::kTileBytes + h * 16384, &tmK, bar(B_KF + ks),
-                        h * 64, j * 128, kvh);
-          if (++ks == C::kStages) { ks = 0; kph ^= 1; }
-          if (!(ok = mbar_wait(bar(B_VE + vs), vph ^ 1, abort_flag, p.status))) break;
-          mbar_arrive_expect_tx(bar(B_VF + vs), C::kTileBytes);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sbase + C::kVOff + vs * C::kTileBytes + h * 16384, &tmV, bar(B_VF + vs),
-                        h * 64, j * 128, kvh);
+  if (warp >= 16) {
+    regs_decrease<C::kRegsOther>();
+    if (warp == C::kWarpProducer) {
+      // ---------------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+          const int u = unit_for_round(r, blockIdx.x, G);
+          if (u >= p.n_units) break;
+          const int qp = p.n_qpairs - 1 - u / p.BH;
+          const int bh = u % p.BH;
+          const int n = unit_kv_tiles(p, qp);
+          if (n == 0) continue;
+          const int kvh = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
+          if (!(ok = mbar_wait(bar(B_QE), (qcount & 1) ^ 1, abort_flag, p.status))) break;
+          ++qcount;
+          mbar_arrive_expect_tx(bar(B_QF), 2 * C::kTileBytes);
+          for (int t = 0; t < 2; ++t)
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + h * 16384, &tmQ, bar(B_QF),
+                          h * 64, qp * 256 + t * 128, bh);
+          for (int j = 0; j < n; ++j) {
+            if (!(ok = mbar_wait(bar(B_KE + ks), kph ^ 1, abort_flag, p.status))) break;
+            mbar_arrive_expect_tx(bar(B_KF + ks), C::kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(sbase + C::kKOff + ks * C::kTileBytes + h * 16384, &tmK, bar(B_KF + ks),
+                          h * 64, j * 128, kvh);
+            if (++ks == C::kStages) { ks = 0; kph ^= 1; }
+            if (!(ok = mbar_wait(bar(B_VE + vs), vph ^ 1, abort_flag, p.status))) break;
+            mbar_arrive_expect_tx(bar(B_VF + vs), C::kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(sbase + C::kVOff + vs * C::kTileBytes + h * 16384, &tmV, bar(B_VF + vs),
+                          h * 64, j * 128, kvh);
+            if (++vs == C::kStages) { vs = 0; vph ^= 1; }
+          }
+        }
+      }
+    } else if (warp == C::kWarpMma) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+        int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
+        int pcount[2] = {0, 0};
+        bool ok = true;
+        // Descriptors of the stage bases; the descriptor of (address + offset) is the
+        // descriptor plus offset >> 4 (the start-address field is the low 14 bits and
+        // every operand lies inside the CTA's shared memory window).
+        const uint64_t dq0 = sdesc_sw128(sbase + C::kQOff, 16, 1024);
+        const uint64_t dk0 = sdesc_sw128(sbase + C::kKOff, 16, 1024);
+        const uint64_t dv0 = sdesc_sw128(sbase + C::kVOff, 16384, 1024);
+        constexpr uint64_t kTileStep = C::kTileBytes >> 4;
+
+        // O_t += P_t V (stage vstage); acc=false overwrites O_t. P_t's keys 0-63 sit in
+        // S_t columns [0,32), keys 64-127 in [64,96).
+        auto issue_pv = [&](int t, int vstage, bool acc) {
+          const uint64_t dv = dv0 + (uint64_t)vstage * kTileStep;
+          const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0);
+          const uint32_t tP = tmem + (t ? C::kColS1 : C::kColS0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tO, tP + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), dv + (uint64_t)(kk * 128),
+                   idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        };
+        auto issue_qk = [&](int t, int kstage) {
+          const uint64_t dq = dq0 + (uint64_t)t * kTileStep;
+          const uint64_t dk = dk0 + (uint64_t)kstage * kTileStep;
+          const uint32_t tS = tmem + (t ? C::kColS1 : C::kColS0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)((kk / 4) * 1024 + (kk % 4) * 2);
+            mma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+        };
+
+        for (int r = 0; ok; ++r) {
+          const int u = unit_for_round(r, blockIdx.x, G);
+          if (u >= p.n_units) break;
+          const int qp = p.n_qpairs - 1 - u / p.BH;
+          const int n = unit_kv_tiles(p, qp);
+          if (n == 0) continue;
+          if (!(ok = mbar_wait(bar(B_QF), qcount & 1, abort_flag, p.status))) break;
+          ++qcount;
+          tc_fence_after();
+          for (int j = 0; j < n && ok; ++j) {
+            if (!(ok = mbar_wait(bar(B_KF + ks), kph, abort_flag, p.status))) break;
+            tc_fence_after();
+            for (int t = 0; t < 2; ++t) {
+              if (j > 0) {
+                if (t == 0) {
+                  if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
+                }
+                if (!(ok = mbar_wait(bar(B_PF + t), pcount[t] & 1, abort_flag, p.status))) break;
+                ++pcount[t];
+                tc_fence_after();
+                issue_pv(t, vs, j > 1);
+                if (t == 1) {
+                  mma_commit(bar(B_VE + vs));
+                  if (++vs == C::kStages) { vs = 0; vph ^= 1; }
+                }
+              }
+              issue_qk(t, ks);
+              mma_commit(bar(B_SF + t));
+            }
+            if (!ok) break;
+            mma_commit(bar(B_KE + ks));
+            if (++ks == C::kStages) { ks = 0; kph ^= 1; }
+          }
+          if (!ok) break;
+          mma_commit(bar(B_QE));
+          // last P.V of the unit
+          if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
+          for (int t = 0; t < 2; ++t) {
+            if (!(ok = mbar_wait(bar(B_PF + t), pcount[t] & 1, abort_flag, p.status))) break;
+            ++pcount[t];
+            tc_fence_after();
+            issue_pv(t, vs, n > 1);
+            mma_commit(bar(B_OD + t));
+          }
+          if (!ok) break;
+          mma_commit(bar(B_VE + vs));
           if (++vs == C::kStages) { vs = 0; vph ^= 1; }
         }
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
-      int pcount[2] = {0, 0};
-      bool ok = true;
-
-      // O_t += P_t V (stage vstage); acc=false overwrites O_t
-      auto issue_pv = [&](int t, int vstage, bool acc) {
-        const uint32_t vaddr = sbase + C::kVOff + vstage * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + (t ? C::kColO1 : C::kColO0), tmem + (t ? C::kColS1 : C::kColS0) + kk * 8, sdesc_sw128(vaddr + kk * 2048, 16384, 1024),
-                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
-      };
-      auto issue_qk = [&](int t, int kstage) {
-        const uint32_t qaddr = sbase + C::kQOff + t * C::kTileBytes;
-        const uint32_t kaddr = sbase + C::kKOff + kstage * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          mma_ss(tmem + (t ? C::kColS1 : C::kColS0), sdesc_sw128(qaddr + off, 16, 1024),
-                 sdesc_sw128(kaddr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-      };
-
-      for (int r = 0; ok; ++r) {
-        const int u = unit_for_round(r, blockIdx.x, G);
-        if (u >= p.n_units) break;
-        const int qp = p.n_qpairs - 1 - u / p.BH;
-        const int n = unit_kv_tiles(p, qp);
-        if (n == 0) continue;
-        if (!(ok = mbar_wait(bar(B_QF), qcount & 1, abort_flag, p.status))) break;
-        ++qcount;
-        tc_fence_after();
-        for (int j = 0; j < n && ok; ++j) {
-          if (!(ok = mbar_wait(bar(B_KF + ks), kph, abort_flag, p.status))) break;
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (j > 0) {
-              if (t == 0) {
-                if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
-              }
-              if (!(ok = mbar_wait(bar(B_PF + t), pcount[t] & 1, abort_flag, p.status))) break;
-              ++pcount[t];
-              tc_fence_after();
-              issue_pv(t, vs, j > 1);
-              if (t == 1) {
-                mma_commit(bar(B_VE + vs));
-                if (++vs == C::kStages) { vs = 0; vph ^= 1; }
-              }
-            }
-            issue_qk(t, ks);
-            mma_commit(bar(B_SF + t));
-          }
-          if (!ok) break;
-          mma_commit(bar(B_KE + ks));
-          if (++ks == C::kStages) { ks = 0; kph ^= 1; }
-        }
-        if (!ok) break;
-        mma_commit(bar(B_QE));
-        // last P.V of the unit
-        if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
-        for (int t = 0; t < 2; ++t) {
-          if (!(ok = mbar_wait(bar(B_PF + t), pcount[t] & 1, abort_flag, p.status))) break;
-          ++pcount[t];
-          tc_fence_after();
-          issue_pv(t, vs, n > 1);
-          mma_commit(bar(B_OD + t));
-        }
-        if (!ok) break;
-        mma_commit(bar(B_VE + vs));
-        if (++vs == C::kStages) { vs = 0; vph ^= 1; }
-      }
-    }
-  }
   } else {
     regs_increase<C::kRegsSoftmax>();
-    // ------------------------------------------------------------------ softmax warpgroups
-    const int t = warp / 4;                 // which Q tile of the unit
+    // ------------------------------------------------------------------ softmax
+    const int wg = warp / 4;
+    const int t = wg >> 1;                  // which Q tile of the unit
+    const int h = wg & 1;                   // which half of the 128 keys
     const int wq = warp % 4;                // warp's TMEM lane quarter
     const int r = wq * 32 + lane;           // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0);
-    const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0);
+    const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0) + 64 * h;
+    const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0) + (D / 2) * h;
+    const uint32_t pair_bar = 1 + 4 * t + wq;  // the two warps that share these rows
+    float* xch_mine = xch + ((t * 2) * 2 + h) * 128 + r;        // + parity * 256
+    const float* xch_other = xch + ((t * 2) * 2 + (h ^ 1)) * 128 + r;
+    float* xl_mine = xl + (t * 2 + h) * 128 + r;
+    const float* xl_other = xl + (t * 2 + (h ^ 1)) * 128 + r;
     const float c = p.scale_log2;
     int scount = 0, ocount = 0;
     bool ok = true;
+    // The two warps of a row pair meet at a named barrier once per key tile and once per
+    // epilogue. A warp that stops on an abort does one non-blocking arrival on its way
+    // out, which releases a partner already waiting; a partner not yet there sees the
+    // abort flag before the barrier and stops too.
+    auto pair_sync = [&]() -> bool {
+      if (*abort_flag) return false;
+      named_bar_sync(pair_bar, 64);
+      return true;
+    };
 
     for (int rr = 0; ok; ++rr) {
       const int u = unit_for_round(rr, blockIdx.x, G);
@@ -330,13 +377,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const long long row0 = (long long)qp * 256 + t * 128;  // first row of this tile
       const long long row = row0 + r;
       const bool row_valid = row < p.Nq;
-      float* orow = p.o + ((long long)bh * p.Nq + row) * D;
+      float* orow = p.o + ((long long)bh * p.Nq + row) * D + (D / 2) * h;
 
       if (n == 0) {
         if (row_valid) {
           float4* o4 = reinterpret_cast<float4*>(orow);
-          for (int i = 0; i < D / 4; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          p.lse[(long long)bh * p.Nq + row] = -INFINITY;
+          for (int i = 0; i < D / 8; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (h == 0) p.lse[(long long)bh * p.Nq + row] = -INFINITY;
         }
         continue;
       }
@@ -351,64 +398,83 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
 
       float m = -INFINITY;  // running maximum (log2 units) used for the exponent
-      float l = 0.f;        // running denominator
+      float l = 0.f;        // this half's running denominator
 
       for (int j = 0; j < n; ++j) {
         ok = mbar_wait(bar(B_SF + t), scount & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
+        const int par = scount & 1;
         ++scount;
         tc_fence_after();
 
-        uint32_t s[4][32];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, s[q4]);
+        uint32_t s[2][32];
+        tmem_ld32(tS, s[0]);
+        tmem_ld32(tS + 32, s[1]);
         tmem_ld_wait(s[0]);
         reg_fence(s[1]);
-        reg_fence(s[2]);
-        reg_fence(s[3]);
 
-        const long long kbase = (long long)j * 128;
-        const bool need_mask = (kbase + 127 > lim_tile);
-        // keys with local column <= climit are visible for this row
-        long long cl = lim_row - kbase;
-        const int climit = cl < -1 ? -1 : (cl > 127 ? 127 : (int)cl);
+        const long long kbase = (long long)j * 128 + 64 * h;
+        const bool need_mask = ((long long)j * 128 + 127 > lim_tile);
+        // this half's keys with local column <= climit are visible for this row
+        const long long cl = lim_row - kbase;
+        const int climit = cl < -1 ? -1 : (cl > 63 ? 63 : (int)cl);
 
-        if (need_mask) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (q4 * 32 + i > climit) s[q4][i] = __float_as_uint(-INFINITY);
-        }
-        float mx;
-        {
-          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            m0 = fmax3(m0, __uint_as_float(s[0][2 * i]), __uint_as_float(s[0][2 * i + 1]));
-            m1 = fmax3(m1, __uint_as_float(s[1][2 * i]), __uint_as_float(s[1][2 * i + 1]));
-            m2 = fmax3(m2, __uint_as_float(s[2][2 * i]), __uint_as_float(s[2][2 * i + 1]));
-            m3 = fmax3(m3, __uint_as_float(s[3][2 * i]), __uint_as_float(s[3][2 * i + 1]));
+        float m_new, alpha, sum;
+        // both warps of a row pair take the same branch (same rows, same m)
+        if (__all_sync(0xffffffffu, !need_mask && m != -INFINITY)) {
+          // Common case: exponentiate against the current running maximum while the tile
+          // maximum is reduced alongside; the maximum only moves when a row's tile maximum
+          // exceeds it by more than 8 (log2 units), and then the warp redoes P.
+          float mx;
+          sum = softmax_half<false, true, C::kPolyFrom>(s, tS, c, m, climit, &mx);
+          xch_mine[par * 256] = mx;
+          if (!(ok = pair_sync())) break;
+          mx = fmaxf(mx, xch_other[par * 256]);
+          const float m_tile = mx * c;
+          const bool grow = m_tile > m + 8.0f;
+          m_new = grow ? m_tile : m;
+          alpha = grow ? ex2_approx(m - m_new) : 1.f;
+          if (__any_sync(0xffffffffu, grow)) {
+            tmem_st_wait();  // the first P stores land before they are overwritten
+            sum = softmax_half<false, false, C::kPolyFrom>(s, tS, c, m_new, climit, nullptr);
           }
-          mx = fmax3(m0, m1, fmaxf(m2, m3));
+        } else {
+          float mx = -INFINITY;
+          {
+            float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float v0 = (2 * i > climit) ? -INFINITY : __uint_as_float(s[0][2 * i]);
+              const float v1 = (2 * i + 1 > climit) ? -INFINITY : __uint_as_float(s[0][2 * i + 1]);
+              const float v2 = (32 + 2 * i > climit) ? -INFINITY : __uint_as_float(s[1][2 * i]);
+              const float v3 =
+                  (33 + 2 * i > climit) ? -INFINITY : __uint_as_float(s[1][2 * i + 1]);
+              m0 = fmax3(m0, v0, v1);
+              m1 = fmax3(m1, v2, v3);
+            }
+            mx = fmaxf(m0, m1);
+          }
+          xch_mine[par * 256] = mx;
+          if (!(ok = pair_sync())) break;
+          mx = fmaxf(mx, xch_other[par * 256]);
+          const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * c;
+          m_new = (m_tile > m + 8.0f) ? m_tile : m;
+          // 1 when unchanged (also when both are -inf), 0 when m was -inf
+          alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          sum = need_mask ? softmax_half<true, false, 16>(s, tS, c, m_use, climit, nullptr)
+                          : softmax_half<false, false, C::kPolyFrom>(s, tS, c, m_use, climit,
+                                                                     nullptr);
         }
-        const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * c;
-        const float m_new = (m_tile > m + 8.0f) ? m_tile : m;
-        // 1 when unchanged (also when both are -inf), 0 when m was -inf
-        const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-
-        float sum = need_mask ? softmax_tile<true>(s, tS, c, m_use, climit)
-                              : softmax_tile<false>(s, tS, c, m_use, climit);
         l = l * alpha + sum;
 
-        // rescale this warp's rows of O when any of them moved its maximum
+        // rescale this thread's half of its row of O when its maximum moved
         const bool moved = (m_new != m) && (j > 0);
         if (__any_sync(0xffffffffu, moved)) {
           const float a = moved ? alpha : 1.f;
 #pragma unroll
-          for (int q4 = 0; q4 < D / 32; ++q4) {
+          for (int q4 = 0; q4 < D / 64; ++q4) {
             uint32_t ov[32];
             tmem_ld32(tO + q4 * 32, ov);
             tmem_ld_wait(ov);
@@ -431,10 +497,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!ok) break;
       ++ocount;
       tc_fence_after();
-      const bool nonempty = l > 0.f;
-      const float inv_l = nonempty ? 1.f / l : 0.f;
+      *xl_mine = l;
+      if (!(ok = pair_sync())) break;
+      const float l_row = l + *xl_other;
+      const bool nonempty = l_row > 0.f;
+      const float inv_l = nonempty ? 1.f / l_row : 0.f;
 #pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) {
+      for (int q4 = 0; q4 < D / 64; ++q4) {
         uint32_t ov[32];
         tmem_ld32(tO + q4 * 32, ov);
         tmem_ld_wait(ov);
@@ -462,11 +531,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      if (row_valid) {
+      if (row_valid && h == 0) {
         float lse;
         if (nonempty) {
           float lg;
-          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
+          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l_row));
           lse = (m + lg) * 0.69314718055994530942f;
         } else {
           lse = -INFINITY;
@@ -475,6 +544,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       tc_fence_before();
     }
+    if (!ok) named_bar_arrive(pair_bar, 64);
   }
 
   // ---------------------------------------------------------------------- teardown
@@ -483,19 +553,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __syncthreads();
   if (*abort_flag) {
     // let in-flight tensor-core work and copies land before TMEM is freed
-    if (warp == 9 && lane == 0) {
+    if (warp == C::kWarpMma && lane == 0) {
       mma_commit(bar(B_DRAIN));
       volatile int dummy = 0;
       mbar_wait(bar(B_DRAIN), 0, &dummy, p.status);
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == C::kWarpProducer && lane == 0) {
       const unsigned long long t0 = globaltimer_ns();
       while (globaltimer_ns() - t0 < 200000ull) {
       }
     }
     __syncthreads();
   }
-  if (warp == 9) {
+  if (warp == C::kWarpMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

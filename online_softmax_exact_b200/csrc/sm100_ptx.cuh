@@ -17,8 +17,12 @@ enum : unsigned {
 };
 
 // Wait limit for any mbarrier: far above any legitimate wait (one tile of work is
-// microseconds), far below anything that looks like a hang.
-constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+// microseconds), far below anything that looks like a hang. Counted in SM clock cycles
+// (cheap to read): 2^31 cycles is about 1.1 s at 1.9 GHz.
+constexpr long long kWaitLimitCycles = 1ll << 31;
+// Longest time a waiting thread stays parked in one try_wait before it re-checks the
+// abort flag and the limit; it wakes as soon as the phase completes.
+constexpr uint32_t kSuspendHintNs = 200000u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -54,25 +58,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete. Returns false if the
-// CTA-wide abort flag is raised or the time limit passes (which raises the flag and
-// records kDevTimeout in *status). Callers stop their role on false.
+// Bounded wait for the phase with the given parity to complete. The thread is parked
+// in try_wait (woken when the phase completes); between parks it checks the CTA-wide
+// abort flag and the cycle limit. Returns false if the flag is raised or the limit
+// passes (which raises the flag and records kDevTimeout in *status). Callers stop
+// their role on false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned* status) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       *abort_flag = 1;
       atomicOr(status, kDevTimeout);
       return false;
@@ -110,6 +116,16 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Arrive at a named barrier without waiting (releases peers that wait on it).
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Register reallocation between warpgroups (all 128 threads of a warpgroup execute it).
