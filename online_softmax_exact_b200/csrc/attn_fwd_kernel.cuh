@@ -86,7 +86,9 @@ struct FwdCfg {
   static constexpr int kRegsOther = 64;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
   // In each 16-pair chunk of a half row, pairs i >= kPolyFrom use the FMA-pipe 2^x.
-  static constexpr int kPolyFrom = 16;
+  // d = 64 needs twice the exponentials per tensor-core FLOP of d = 128, so it hands a
+  // quarter of them to the FMA pipe; at d = 128 the exp unit keeps up on its own.
+  static constexpr int kPolyFrom = (D == 64) ? 12 : 16;
 };
 
 __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
@@ -117,6 +119,7 @@ __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP,
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   const uint64_t C2 = f2_pack(c, c);
   const uint64_t NM2 = f2_pack(-m_use, -m_use);
+  const Exp2PolyConsts pk_consts;
 #pragma unroll
   for (int q2 = 0; q2 < 2; ++q2) {
     uint32_t pk[16];
@@ -130,14 +133,15 @@ __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP,
           mx0 = fmax3(mx0, s0, s1);
       }
       float x0, x1, e0, e1;
-      f2_unpack(f2_fma(f2_pack(s0, s1), C2, NM2), x0, x1);
+      const uint64_t X = f2_fma(f2_pack(s0, s1), C2, NM2);
+      f2_unpack(X, x0, x1);
       if (kMasked) {
         if (q2 * 32 + 2 * i > climit) x0 = -INFINITY;
         if (q2 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
         e0 = ex2_approx(x0);
         e1 = ex2_approx(x1);
       } else if (i >= kPolyFrom) {
-        exp2_poly_pair(x0, x1, e0, e1);
+        exp2_poly_pair(X, pk_consts, e0, e1);
       } else {
         e0 = ex2_approx(x0);
         e1 = ex2_approx(x1);

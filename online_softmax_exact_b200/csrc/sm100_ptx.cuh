@@ -335,24 +335,33 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
 // polynomial (coefficients fitted by exp2_poly_fit.py for minimum relative error:
 // 1.03e-4 at most), and n added to the exponent field. Inputs below -125 give 2^-125
 // or so instead of a smaller value; callers only pass rows whose denominator is >= 1.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t X = f2_pack(x0, x1);
-  const uint64_t SH = f2_pack(kShift, kShift);
-  const uint64_t J = f2_add(X, SH);       // kShift + round(x): n in the low mantissa bits
-  const uint64_t R = f2_sub(J, SH);       // round(x) as a float
-  const uint64_t F = f2_sub(X, R);        // f in [-1/2, 1/2]
-  uint64_t P = f2_fma(f2_pack(kExp2C3, kExp2C3), F, f2_pack(kExp2C2, kExp2C2));
-  P = f2_fma(P, F, f2_pack(kExp2C1, kExp2C1));
-  P = f2_fma(P, F, f2_pack(1.0f, 1.0f));
-  float p0, p1, j0, j1;
-  f2_unpack(P, p0, p1);
-  f2_unpack(J, j0, j1);
-  // (kShift + n) << 23 leaves exactly n << 23 in 32 bits
-  y0 = __uint_as_float(__float_as_uint(j0) * 8388608u + __float_as_uint(p0));
-  y1 = __uint_as_float(__float_as_uint(j1) * 8388608u + __float_as_uint(p1));
+// The pair stays packed (f32x2 arithmetic) from the input to the exponent add.
+struct Exp2PolyConsts {
+  uint64_t shift, c3, c2, c1, one;
+  __device__ __forceinline__ Exp2PolyConsts()
+      : shift(f2_pack(12582912.0f, 12582912.0f)),  // 1.5 * 2^23
+        c3(f2_pack(kExp2C3, kExp2C3)),
+        c2(f2_pack(kExp2C2, kExp2C2)),
+        c1(f2_pack(kExp2C1, kExp2C1)),
+        one(f2_pack(1.0f, 1.0f)) {}
+};
+
+__device__ __forceinline__ void exp2_poly_pair(uint64_t X, const Exp2PolyConsts& k, float& y0,
+                                               float& y1) {
+  float x0, x1;
+  f2_unpack(X, x0, x1);
+  const uint64_t Xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t J = f2_add(Xc, k.shift);           // shift + round(x): n in the low bits
+  const uint64_t F = f2_sub(Xc, f2_sub(J, k.shift));  // f = x - round(x) in [-1/2, 1/2]
+  uint64_t P = f2_fma(k.c3, F, k.c2);
+  P = f2_fma(P, F, k.c1);
+  P = f2_fma(P, F, k.one);
+  uint32_t p0, p1, j0, j1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(P));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(J));
+  // (shift + n) << 23 leaves exactly n << 23 in 32 bits
+  y0 = __uint_as_float(j0 * 8388608u + p0);
+  y1 = __uint_as_float(j1 * 8388608u + p1);
 }
 
 }  // namespace osx
