@@ -461,6 +461,27 @@ def run_ours(args, w) -> int:
     merge_gbs = mbytes / (t_merge * 1e-3) / 1e9 if t_merge > 0 else None
     attn_single = partial_flops_per_step * n_iso / (t_part1 * 1e-3) / 1e12 if t_part1 else None
 
+    # ---- the same ring step with the fused running merge (attn_fwd_partial_acc): no
+    # partial buffers, no merge launches
+    def step_fused():
+        ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
+                       stream=stream, n_streams=args.streams, fused_merge=True)
+
+    for _ in range(3):
+        step_fused()
+    torch.cuda.synchronize()
+    n_fused = max(3, min(args.steps, 30))
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(n_fused):
+        step_fused()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ms_fused = max_over_ranks(f0.elapsed_time(f1), dev) / n_fused
+    if osx.attn_device_status() != osx.ATTN_OK:
+        raise RuntimeError("device-side wait ran out of time in the fused ring step")
+
     # ---- end to end through the public API with pinned host buffers
     e2e = run_e2e(args, w, q_h, k_h, v_h, dev, out, ws, world)
 
@@ -492,6 +513,12 @@ def run_ours(args, w) -> int:
                   "busy_ms": t_merge, "summed_launch_ms": sum_merge,
                   "timing": f"the same ring step on one stream, {n_iso} steps after the timed "
                             "region; algorithmic bytes / CUDA-event time of the merge launches"},
+        "fused_running_merge": {
+            "value": w.flops * world / (ms_fused * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms_fused, "steps": n_fused,
+            "what": "the same ring step with each query chunk's partials folded into one "
+                    "running (O, LSE) accumulator by attn_fwd_partial_acc: 36 attention "
+                    "launches, no merge launches, no partial buffers"},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),

@@ -111,6 +111,29 @@ attn_status_t attn_fwd_partial(const void* q, const void* k_chunk, const void* v
                                float scale, void* stream);
 
 /*
+ * attn_fwd_partial_acc - attn_fwd_partial fused with the merge: o_acc and lse_acc
+ * hold, on entry, a normalised partial result over keys disjoint from this chunk
+ * (LSE = -inf with O = 0 where no key has been seen yet), and on exit the
+ * combination of that partial with this chunk's, by the same log-sum-exp rule as
+ * attn_merge. This is the running update a Ring Attention device applies at each
+ * ring step ("Ring Attention with Blockwise Parallel Transformers", section 3) and the
+ * rescale of the online softmax ("FlashAttention by hand", paragraphs on the running
+ * statistics and rescaling) applied at chunk granularity; it needs no buffer for the
+ * chunk's own partial and no separate merge launch. A chunk none of whose keys is
+ * visible to a row leaves that row unchanged.
+ *
+ *   o_acc, lse_acc  device, fp32 [B][Hq][Nq][d] and [B][Hq][Nq], read and written
+ *   other arguments exactly as for attn_fwd_partial.
+ * Successive calls on one accumulator must be ordered (one stream); calls on
+ * different accumulators may run concurrently.
+ */
+attn_status_t attn_fwd_partial_acc(const void* q, const void* k_chunk, const void* v_chunk,
+                                   float* o_acc, float* lse_acc, int B, int Hq, int Hkv,
+                                   int64_t Nq, int64_t Nkv, int64_t q_ld, int64_t kv_ld,
+                                   int64_t q_off, int64_t kv_off, int d, int causal,
+                                   float scale, void* stream);
+
+/*
  * attn_merge - combine partial results computed over disjoint key sets
  * (ATTENTION2D, section 3: fragment-local statistics normalised and summed in
  * stages; section 2: the combination is commutative and associative, so no
@@ -148,6 +171,16 @@ attn_status_t attn_device_status(void* stream, int reset);
  * count = 0 disarms. Not thread-safe; for tests only.
  */
 attn_status_t attn_debug_inject(int status, int count);
+
+/*
+ * attn_debug_wait_timeout - failure-path check for tests: launches one tiny kernel
+ * whose single waiting thread waits, through the same bounded mbarrier wait the
+ * attention kernel uses, on a barrier that nothing arrives on, with a limit of
+ * limit_cycles SM clock cycles (1 .. 2^31). The wait runs out, the kernel records
+ * ATTN_ERR_TIMEOUT in the device status word (see attn_device_status) and returns;
+ * the device stays usable. Nothing traps or faults.
+ */
+attn_status_t attn_debug_wait_timeout(int64_t limit_cycles, void* stream);
 
 /* Number of CUDA kernels this library has launched in this process (all devices). */
 uint64_t attn_launch_count(void);

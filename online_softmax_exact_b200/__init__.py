@@ -3,7 +3,8 @@
 A thin binding over the C ABI of ``libattn.so`` (``include/attn.h``): the functions
 here check and marshal torch tensors and call the entry point of the same name.
 All arithmetic runs in the library's CUDA kernels; torch provides device memory and
-streams only. If the library is missing, importing this package raises.
+streams only. The library is loaded on first use; if it is missing or out of date
+that first call raises (there is no fallback implementation).
 """
 
 from __future__ import annotations
@@ -24,18 +25,23 @@ from ._abi import (
     load,
 )
 
-_lib = load()
+_lib_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libattn.so (loaded on first use)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = load()
+    return _lib_handle
 
 __all__ = [
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA",
     "ATTN_ERR_TIMEOUT", "ATTN_ERR_INJECTED", "ATTN_MAX_MERGE_PARTS", "AttnError",
-    "attn_fwd", "attn_fwd_partial", "attn_merge", "attn_device_status", "attn_debug_inject",
+    "attn_fwd", "attn_fwd_partial", "attn_fwd_partial_acc", "attn_merge", "attn_device_status", "attn_debug_inject",
     "attn_launch_count", "attn_status_string", "attn_version", "lib",
+    "attn_debug_wait_timeout",
 ]
-
-
-def lib() -> ctypes.CDLL:
-    return _lib
 
 
 def _stream_handle(device: torch.device, stream) -> int:
@@ -59,15 +65,15 @@ def _need(t: torch.Tensor, dtype, name: str) -> None:
 
 
 def attn_status_string(status: int) -> str:
-    return _lib.attn_status_string(int(status)).decode()
+    return lib().attn_status_string(int(status)).decode()
 
 
 def attn_version() -> int:
-    return int(_lib.attn_version())
+    return int(lib().attn_version())
 
 
 def attn_launch_count() -> int:
-    return int(_lib.attn_launch_count())
+    return int(lib().attn_launch_count())
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
@@ -91,10 +97,43 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     _need(o, torch.float32, "o")
     _need(lse, torch.float32, "lse")
-    st = _lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+    st = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        B, Hq, Hkv, N, d, int(bool(causal)), float(scale),
                        _stream_handle(q.device, stream))
     _check(st, "attn_fwd")
+    return o, lse
+
+
+def _partial(entry: str, q, k, v, q_start, q_len, kv_start, kv_len, causal, scale, q_off,
+             kv_off, o, lse, stream, alloc: bool):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, Lq, d = q.shape
+    Hkv, Lkv = k.shape[1], k.shape[2]
+    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Hkv, Lkv, d] matching q")
+    if not (0 <= q_start and q_start + q_len <= Lq and 0 <= kv_start and kv_start + kv_len <= Lkv):
+        raise ValueError("chunk outside its parent tensor")
+    if scale is None:
+        scale = d ** -0.5
+    q_off = q_start if q_off is None else q_off
+    kv_off = kv_start if kv_off is None else kv_off
+    if o is None or lse is None:
+        if not alloc:
+            raise ValueError("the accumulator (o, lse) must be given")
+        o = torch.empty((B, Hq, q_len, d), dtype=torch.float32, device=q.device) if o is None else o
+        lse = torch.empty((B, Hq, q_len), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(o, torch.float32, "o")
+    _need(lse, torch.float32, "lse")
+    if o.shape != (B, Hq, q_len, d) or lse.shape != (B, Hq, q_len):
+        raise ValueError("o / lse must be [B, Hq, q_len, d] / [B, Hq, q_len]")
+    es = q.element_size()
+    st = getattr(lib(), entry)(
+        q.data_ptr() + q_start * d * es, k.data_ptr() + kv_start * d * es,
+        v.data_ptr() + kv_start * d * es, o.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+        q_len, kv_len, Lq, Lkv, int(q_off), int(kv_off), d, int(bool(causal)), float(scale),
+        _stream_handle(q.device, stream))
+    _check(st, entry)
     return o, lse
 
 
@@ -110,32 +149,18 @@ def attn_fwd_partial(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, q_sta
     (q_off = q_start, kv_off = kv_start). Returns the normalised partial
     (O fp32 [B,Hq,q_len,d], LSE fp32 [B,Hq,q_len]).
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, torch.bfloat16, n)
-    B, Hq, Lq, d = q.shape
-    Hkv, Lkv = k.shape[1], k.shape[2]
-    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != d:
-        raise ValueError("k and v must be [B, Hkv, Lkv, d] matching q")
-    if not (0 <= q_start and q_start + q_len <= Lq and 0 <= kv_start and kv_start + kv_len <= Lkv):
-        raise ValueError("chunk outside its parent tensor")
-    if scale is None:
-        scale = d ** -0.5
-    q_off = q_start if q_off is None else q_off
-    kv_off = kv_start if kv_off is None else kv_off
-    if o is None:
-        o = torch.empty((B, Hq, q_len, d), dtype=torch.float32, device=q.device)
-    if lse is None:
-        lse = torch.empty((B, Hq, q_len), dtype=torch.float32, device=q.device)
-    _need(o, torch.float32, "o")
-    _need(lse, torch.float32, "lse")
-    es = q.element_size()
-    st = _lib.attn_fwd_partial(
-        q.data_ptr() + q_start * d * es, k.data_ptr() + kv_start * d * es,
-        v.data_ptr() + kv_start * d * es, o.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
-        q_len, kv_len, Lq, Lkv, int(q_off), int(kv_off), d, int(bool(causal)), float(scale),
-        _stream_handle(q.device, stream))
-    _check(st, "attn_fwd_partial")
-    return o, lse
+    return _partial("attn_fwd_partial", q, k, v, q_start, q_len, kv_start, kv_len, causal,
+                    scale, q_off, kv_off, o, lse, stream, alloc=True)
+
+
+def attn_fwd_partial_acc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, q_start: int,
+                         q_len: int, kv_start: int, kv_len: int, causal: bool,
+                         o: torch.Tensor, lse: torch.Tensor, scale: float | None = None,
+                         q_off: int | None = None, kv_off: int | None = None, stream=None):
+    """Like :func:`attn_fwd_partial`, folding the chunk's result into the accumulator
+    (o, lse) in place (log-sum-exp merge). Returns (o, lse)."""
+    return _partial("attn_fwd_partial_acc", q, k, v, q_start, q_len, kv_start, kv_len,
+                    causal, scale, q_off, kv_off, o, lse, stream, alloc=False)
 
 
 def attn_merge(o_parts, lse_parts, *, o: torch.Tensor | None = None,
@@ -164,7 +189,7 @@ def attn_merge(o_parts, lse_parts, *, o: torch.Tensor | None = None,
     _need(lse, torch.float32, "lse")
     optr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in o_parts])
     lptr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in lse_parts])
-    st = _lib.attn_merge(optr, lptr, n, o.data_ptr(), lse.data_ptr(), rows, d,
+    st = lib().attn_merge(optr, lptr, n, o.data_ptr(), lse.data_ptr(), rows, d,
                          _stream_handle(ref.device, stream))
     _check(st, "attn_merge")
     return o, lse
@@ -173,8 +198,15 @@ def attn_merge(o_parts, lse_parts, *, o: torch.Tensor | None = None,
 def attn_device_status(stream=None, reset: bool = False) -> int:
     """Synchronise the stream; return ATTN_OK or ATTN_ERR_TIMEOUT (device-side record)."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    return int(_lib.attn_device_status(_stream_handle(dev, stream), int(bool(reset))))
+    return int(lib().attn_device_status(_stream_handle(dev, stream), int(bool(reset))))
 
 
 def attn_debug_inject(status: int, count: int) -> None:
-    _check(_lib.attn_debug_inject(int(status), int(count)), "attn_debug_inject")
+    _check(lib().attn_debug_inject(int(status), int(count)), "attn_debug_inject")
+
+
+def attn_debug_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Launch the failure-path check kernel (a bounded wait that must run out)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib().attn_debug_wait_timeout(int(limit_cycles), _stream_handle(dev, stream)),
+           "attn_debug_wait_timeout")

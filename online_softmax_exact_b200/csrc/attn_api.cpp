@@ -40,7 +40,7 @@ attn_status_t take_injected() {
 attn_status_t check_and_launch(const void* q, const void* k, const void* v, float* o, float* lse,
                                int B, int Hq, int Hkv, int64_t Nq, int64_t Nkv, int64_t q_ld,
                                int64_t kv_ld, int64_t q_off, int64_t kv_off, int d, int causal,
-                               float scale, void* stream) {
+                               float scale, void* stream, int accumulate) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (Nq < 1 || Nkv < 1 || q_ld < Nq || kv_ld < Nkv || q_off < 0 || kv_off < 0)
@@ -87,6 +87,7 @@ attn_status_t check_and_launch(const void* q, const void* k, const void* v, floa
   a.d = d;
   a.causal = causal;
   a.scale = scale;
+  a.accumulate = accumulate;
   return static_cast<attn_status_t>(osx::launch_fwd(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -110,7 +111,8 @@ int attn_version(void) { return (1 << 16) | 0; }
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, float* o, float* lse, int B,
                        int Hq, int Hkv, int64_t N, int d, int causal, float scale, void* stream) {
-  return check_and_launch(q, k, v, o, lse, B, Hq, Hkv, N, N, N, N, 0, 0, d, causal, scale, stream);
+  return check_and_launch(q, k, v, o, lse, B, Hq, Hkv, N, N, N, N, 0, 0, d, causal, scale, stream,
+                          0);
 }
 
 attn_status_t attn_fwd_partial(const void* q, const void* k_chunk, const void* v_chunk,
@@ -118,7 +120,16 @@ attn_status_t attn_fwd_partial(const void* q, const void* k_chunk, const void* v
                                int64_t Nkv, int64_t q_ld, int64_t kv_ld, int64_t q_off,
                                int64_t kv_off, int d, int causal, float scale, void* stream) {
   return check_and_launch(q, k_chunk, v_chunk, o_part, lse_part, B, Hq, Hkv, Nq, Nkv, q_ld, kv_ld,
-                          q_off, kv_off, d, causal, scale, stream);
+                          q_off, kv_off, d, causal, scale, stream, 0);
+}
+
+attn_status_t attn_fwd_partial_acc(const void* q, const void* k_chunk, const void* v_chunk,
+                                   float* o_acc, float* lse_acc, int B, int Hq, int Hkv,
+                                   int64_t Nq, int64_t Nkv, int64_t q_ld, int64_t kv_ld,
+                                   int64_t q_off, int64_t kv_off, int d, int causal, float scale,
+                                   void* stream) {
+  return check_and_launch(q, k_chunk, v_chunk, o_acc, lse_acc, B, Hq, Hkv, Nq, Nkv, q_ld, kv_ld,
+                          q_off, kv_off, d, causal, scale, stream, 1);
 }
 
 attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts,
@@ -159,6 +170,12 @@ attn_status_t attn_debug_inject(int status, int count) {
   g_inject_status = status;
   g_inject_count = count;
   return ATTN_OK;
+}
+
+attn_status_t attn_debug_wait_timeout(int64_t limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 31)) return ATTN_ERR_INVALID_ARG;
+  return static_cast<attn_status_t>(
+      osx::launch_wait_probe(limit_cycles, static_cast<cudaStream_t>(stream)));
 }
 
 uint64_t attn_launch_count(void) { return osx::launch_count(); }

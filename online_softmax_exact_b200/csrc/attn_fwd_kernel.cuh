@@ -27,7 +27,9 @@
 //     same base. In the common case the exponentials are computed against the current
 //     m while the tile maximum is reduced alongside, and redone only if m moves; when
 //     m moves the threads rescale their halves of O in TMEM;
-//   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32.
+//   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32; in accumulate mode
+//     the result is first combined with the normalised partial (O_acc, LSE_acc) already
+//     in o/lse by the log-sum-exp rule of the merge (weights e^(LSE - max LSE)).
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [384,384+D). Half h of P_t (bf16 pairs) overwrites S_t columns [64h, 64h+32),
@@ -55,6 +57,7 @@ struct FwdParams {
   int n_units;         // n_qpairs * BH
   int n_kv_tiles;      // ceil(Nkv / 128)
   int o_vec8;          // O is 32-byte aligned: store rows with 256-bit stores
+  int accumulate;      // o/lse hold a partial over other keys: fold this chunk into it
 };
 
 template <int D>
@@ -384,7 +387,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float* orow = p.o + ((long long)bh * p.Nq + row) * D + (D / 2) * h;
 
       if (n == 0) {
-        if (row_valid) {
+        // no key of this chunk is visible to the unit: the result is empty (O = 0,
+        // LSE = -inf), and folding an empty result into an accumulator changes nothing
+        if (row_valid && !p.accumulate) {
           float4* o4 = reinterpret_cast<float4*>(orow);
           for (int i = 0; i < D / 8; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (h == 0) p.lse[(long long)bh * p.Nq + row] = -INFINITY;
@@ -501,11 +506,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!ok) break;
       ++ocount;
       tc_fence_after();
+      // in accumulate mode both threads of the row read the old LSE before the pair
+      // barrier; the new one is written after it
+      float lse_acc = -INFINITY;
+      if (p.accumulate && row_valid) lse_acc = p.lse[(long long)bh * p.Nq + row];
       *xl_mine = l;
       if (!(ok = pair_sync())) break;
       const float l_row = l + *xl_other;
       const bool nonempty = l_row > 0.f;
-      const float inv_l = nonempty ? 1.f / l_row : 0.f;
+      float lse_new = -INFINITY;
+      if (nonempty) {
+        float lg;
+        asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l_row));
+        lse_new = (m + lg) * 0.69314718055994530942f;
+      }
+      // out = a * O_acc + b * O_tmem
+      float a = 0.f, b = nonempty ? 1.f / l_row : 0.f, lse_out = lse_new;
+      if (p.accumulate) {
+        const float M = fmaxf(lse_acc, lse_new);
+        if (M == -INFINITY) {
+          b = 0.f;
+        } else {
+          constexpr float kLog2e = 1.4426950408889634f;
+          const float wa = ex2_approx((lse_acc - M) * kLog2e);  // 0 for an empty accumulator
+          const float wn = ex2_approx((lse_new - M) * kLog2e);
+          const float inv = 1.f / (wa + wn);
+          a = wa * inv;
+          b = nonempty ? wn * inv / l_row : 0.f;
+          float lg;
+          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(wa + wn));
+          lse_out = M + lg * 0.69314718055994530942f;
+        }
+      }
 #pragma unroll
       for (int q4 = 0; q4 < D / 64; ++q4) {
         uint32_t ov[32];
@@ -513,39 +545,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld_wait(ov);
         if (row_valid) {
           float* dst = orow + q4 * 32;
+          float res[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
+          if (a != 0.f) {  // only then is the old accumulator read
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 old = *reinterpret_cast<const float4*>(dst + i);
+              res[i] = fmaf(a, old.x, res[i]);
+              res[i + 1] = fmaf(a, old.y, res[i + 1]);
+              res[i + 2] = fmaf(a, old.z, res[i + 2]);
+              res[i + 3] = fmaf(a, old.w, res[i + 3]);
+            }
+          }
           if (p.o_vec8) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              st_global_v8(dst + 8 * i, __uint_as_float(ov[8 * i]) * inv_l,
-                           __uint_as_float(ov[8 * i + 1]) * inv_l,
-                           __uint_as_float(ov[8 * i + 2]) * inv_l,
-                           __uint_as_float(ov[8 * i + 3]) * inv_l,
-                           __uint_as_float(ov[8 * i + 4]) * inv_l,
-                           __uint_as_float(ov[8 * i + 5]) * inv_l,
-                           __uint_as_float(ov[8 * i + 6]) * inv_l,
-                           __uint_as_float(ov[8 * i + 7]) * inv_l);
+              st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
+                           res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
+                           res[8 * i + 7]);
           } else {
             float4* o4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              o4[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l,
-                                  __uint_as_float(ov[4 * i + 1]) * inv_l,
-                                  __uint_as_float(ov[4 * i + 2]) * inv_l,
-                                  __uint_as_float(ov[4 * i + 3]) * inv_l);
+              o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
           }
         }
       }
-      if (row_valid && h == 0) {
-        float lse;
-        if (nonempty) {
-          float lg;
-          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l_row));
-          lse = (m + lg) * 0.69314718055994530942f;
-        } else {
-          lse = -INFINITY;
-        }
-        p.lse[(long long)bh * p.Nq + row] = lse;
-      }
+      if (row_valid && h == 0) p.lse[(long long)bh * p.Nq + row] = lse_out;
       tc_fence_before();
     }
     if (!ok) named_bar_arrive(pair_bar, 64);

@@ -20,12 +20,15 @@ struct FwdLaunch {
   int d;
   int causal;
   float scale;
+  int accumulate;  // o/lse are an in/out accumulator (see attn_fwd_partial_acc)
 };
 
 // Returns 0 (ATTN_OK) or an attn_status_t failure code.
 int launch_fwd(const FwdLaunch& a, cudaStream_t stream);
 int launch_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts,
                  float* o, float* lse, long long rows, int d, cudaStream_t stream);
+// Launches the failure-path check kernel (a bounded wait that must run out).
+int launch_wait_probe(long long limit_cycles, cudaStream_t stream);
 // Reads (and optionally clears) the device status word of the current device.
 int read_device_status(unsigned* out, int reset);
 uint64_t launch_count();

@@ -16,6 +16,23 @@ namespace osx {
 // out record kDevTimeout here. Read through read_device_status().
 __device__ unsigned g_device_status;
 
+// Failure-path check: one thread waits on an mbarrier that nothing arrives on, through
+// the same bounded wait the attention kernel uses, with a short limit. The wait runs
+// out, records kDevTimeout in the status word and the kernel returns.
+__global__ void wait_probe_kernel(unsigned* status, long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  __shared__ int abort_storage;
+  if (threadIdx.x == 0) {
+    abort_storage = 0;
+    mbar_init(smem_u32(&bar_storage), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait_limit(smem_u32(&bar_storage), 0, &abort_storage, status, limit_cycles);
+  __syncthreads();
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -86,6 +103,7 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
   p.n_units = static_cast<int>(units);
   p.n_kv_tiles = static_cast<int>((a.Nkv + 127) / 128);
   p.o_vec8 = (reinterpret_cast<uintptr_t>(a.o) % 32) == 0 ? 1 : 0;
+  p.accumulate = a.accumulate;
   const int grid = p.n_units < di.num_sms ? p.n_units : di.num_sms;
   attn_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -144,6 +162,16 @@ int launch_merge(const float* const* o_parts, const float* const* lse_parts, int
     case 128: return launch_merge_d<128>(p, *di, stream);
     default: return ATTN_ERR_UNSUPPORTED;
   }
+}
+
+int launch_wait_probe(long long limit_cycles, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != ATTN_OK) return rc;
+  wait_probe_kernel<<<1, 32, 0, stream>>>(di->status, limit_cycles);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return ATTN_OK;
 }
 
 int read_device_status(unsigned* out, int reset) {

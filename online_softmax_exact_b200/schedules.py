@@ -14,7 +14,7 @@ from dataclasses import dataclass
 
 import torch
 
-from . import attn_fwd_partial, attn_merge
+from . import attn_fwd_partial, attn_fwd_partial_acc, attn_merge
 
 
 def chunk_bounds(N: int, n_chunks: int) -> list[tuple[int, int]]:
@@ -114,7 +114,7 @@ class _Streams:
 
 def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None = None,
                    out=None, workspace: Workspace | None = None, stream=None, timer=None,
-                   n_streams: int = 1):
+                   n_streams: int = 1, fused_merge: bool = False):
     """Ring Attention's schedule on one GPU: query chunk i attends the key/value chunks
     of :func:`ring_order` one ring step at a time, then merges its partials.
 
@@ -123,6 +123,10 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
     launch; each chunk's partials and merge stay in order on its stream, and the result
     is joined back into ``stream``. ``timer(kind)``, if given, is entered around every
     launch ("partial" or "merge") with the launching stream as argument.
+    With ``fused_merge`` each query chunk keeps one running (O, LSE) accumulator in the
+    output: the first visited chunk writes it, every later ring step folds its partial
+    into it (``attn_fwd_partial_acc``), as a ring device does; no partial buffers and
+    no merge launches.
     Returns chunk-major (O [P,B,Hq,C,d], LSE [P,B,Hq,C]).
     """
     timer = timer or _NO_TIMER
@@ -134,7 +138,8 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
     slots = max(len(x) for x in order)
     n_streams = max(1, min(n_streams, n_chunks))
     need = slots * n_streams
-    if workspace is None or workspace.o.shape[0] < need or workspace.o.shape[1:] != (B, Hq, C, d):
+    if not fused_merge and (workspace is None or workspace.o.shape[0] < need
+                            or workspace.o.shape[1:] != (B, Hq, C, d)):
         workspace = Workspace.for_shape(need, B, Hq, C, d, q.device)
     main = stream if stream is not None else torch.cuda.current_stream(q.device)
     st = _Streams(main, n_streams, q.device)
@@ -145,6 +150,14 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
         s = st.side[s_idx]
         base = s_idx * slots
         qs, qe = bounds[qi]
+        if fused_merge:
+            for j, kv in enumerate(visit):
+                ks, ke = bounds[kv]
+                fn = attn_fwd_partial if j == 0 else attn_fwd_partial_acc
+                with timer("partial", s):
+                    fn(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                       causal=causal, scale=scale, o=o_out[qi], lse=l_out[qi], stream=s)
+            continue
         if len(visit) == 1:
             # one part: the merge is the identity, so write the result in place
             ks, ke = bounds[visit[0]]
@@ -164,17 +177,19 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
             attn_merge([workspace.o[base + i] for i in range(n)],
                        [workspace.lse[base + i] for i in range(n)],
                        o=o_out[qi], lse=l_out[qi], stream=s)
-    st.join([q, k, v, o_out, l_out, workspace.o, workspace.lse])
+    st.join([q, k, v, o_out, l_out] + ([] if fused_merge else [workspace.o, workspace.lse]))
     return o_out, l_out
 
 
 def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], causal: bool,
                      scale: float | None = None, out=None, workspace: Workspace | None = None,
-                     stream=None, timer=None, n_streams: int = 1):
+                     stream=None, timer=None, n_streams: int = 1, fused_merge: bool = False):
     """ATTENTION2D's query x key/value grid on one GPU: every (query chunk, key/value
     chunk) cell is a partial attention (fragment-local statistics, section 3); each
     query chunk's partials are merged in the order ``merge_orders[i]`` (any order gives
-    the same result, section 2). Returns chunk-major (O, LSE).
+    the same result, section 2). With ``fused_merge`` the cells of a query chunk are
+    folded into one running accumulator in that order instead. Returns chunk-major
+    (O, LSE).
     """
     timer = timer or _NO_TIMER
     B, Hq, N, d = q.shape
@@ -183,8 +198,8 @@ def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], c
     o_out, l_out = _alloc_out(q, n_chunks, out)
     n_streams = max(1, min(n_streams, n_chunks))
     need = n_chunks * n_streams
-    if workspace is None or workspace.o.shape[0] < need or \
-            workspace.o.shape[1:] != (B, Hq, C, d):
+    if not fused_merge and (workspace is None or workspace.o.shape[0] < need
+                            or workspace.o.shape[1:] != (B, Hq, C, d)):
         workspace = Workspace.for_shape(need, B, Hq, C, d, q.device)
     main = stream if stream is not None else torch.cuda.current_stream(q.device)
     st = _Streams(main, n_streams, q.device)
@@ -195,6 +210,14 @@ def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], c
         order = merge_orders[qi]
         if sorted(order) != list(range(n_chunks)):
             raise ValueError("each merge order must be a permutation of the chunk indices")
+        if fused_merge:
+            for j, kv in enumerate(order):
+                ks, ke = bounds[kv]
+                fn = attn_fwd_partial if j == 0 else attn_fwd_partial_acc
+                with timer("partial", s):
+                    fn(q, k, v, q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                       causal=causal, scale=scale, o=o_out[qi], lse=l_out[qi], stream=s)
+            continue
         for kv in range(n_chunks):
             ks, ke = bounds[kv]
             with timer("partial", s):
@@ -206,7 +229,7 @@ def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], c
             attn_merge([workspace.o[base + i] for i in order],
                        [workspace.lse[base + i] for i in order],
                        o=o_out[qi], lse=l_out[qi], stream=s)
-    st.join([q, k, v, o_out, l_out, workspace.o, workspace.lse])
+    st.join([q, k, v, o_out, l_out] + ([] if fused_merge else [workspace.o, workspace.lse]))
     return o_out, l_out
 
 

@@ -52,6 +52,18 @@ def test_ring_32k(osx):
     check_sampled(o, lse, q, k, v, w, 96)
 
 
+def test_ring_32k_fused_merge(osx):
+    from online_softmax_exact_b200.schedules import chunks_to_sequence, ring_attention
+
+    w = get("ring_32k")
+    q, k, v = attention_inputs(w)
+    oc, lc = ring_attention(q.cuda(), k.cuda(), v.cuda(), n_chunks=w.n_chunks, causal=w.causal,
+                            scale=w.scale, fused_merge=True, n_streams=2)
+    assert osx.attn_device_status() == osx.ATTN_OK
+    o, lse = chunks_to_sequence(oc, lc)
+    check_sampled(o, lse, q, k, v, w, 64)
+
+
 def test_gqa_128k_single_pass(osx):
     w = get("gqa_128k")
     q, k, v = attention_inputs(w)
@@ -65,9 +77,11 @@ def test_grid2d_64k_stress(osx):
 
     w = get("grid2d_64k_stress")
     q, k, v = attention_inputs(w)
-    oc, lc = grid2d_attention(q.cuda(), k.cuda(), v.cuda(), n_chunks=w.n_chunks,
-                              merge_orders=grid_merge_orders(w.n_chunks, w.seed),
-                              causal=w.causal, scale=w.scale)
-    assert osx.attn_device_status() == osx.ATTN_OK
-    o, lse = chunks_to_sequence(oc, lc)
-    check_sampled(o, lse, q, k, v, w, 96)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    for fused in (False, True):
+        oc, lc = grid2d_attention(qg, kg, vg, n_chunks=w.n_chunks,
+                                  merge_orders=grid_merge_orders(w.n_chunks, w.seed),
+                                  causal=w.causal, scale=w.scale, fused_merge=fused)
+        assert osx.attn_device_status() == osx.ATTN_OK
+        o, lse = chunks_to_sequence(oc, lc)
+        check_sampled(o, lse, q, k, v, w, 96 if not fused else 48)
