@@ -289,12 +289,15 @@ def run_reference(args, w) -> int:
 METRIC = "attention fwd TFLOP/s and % of bf16 tensor peak on 1 B200; merge HBM GB/s"
 
 
-def workload_config(w, world: int, streams: int | None = None) -> dict:
+def workload_config(w, world: int, streams: int | None = None, batched=None) -> dict:
     return {"workload": f"{w.name}: {w.description}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "N": w.N, "d": w.d, "causal": w.causal, "schedule": w.schedule,
             "n_chunks": w.n_chunks, "global_batch": w.B * world, "seq_len": w.N,
             "parallelism": "single GPU" if world == 1 else f"{world} independent replicas",
             "streams": streams,
+            "launch": None if batched is None else (
+                "one attn_fwd_partial_batch launch for the 36 ring partials, then 7 merges"
+                if batched else "one attn_fwd_partial launch per ring partial, then 7 merges"),
             "l2": "inputs larger than L2 (Q, K, V = 768 MiB per step); no flush"}
 
 
@@ -367,7 +370,7 @@ def run_ours(args, w) -> int:
     dev = torch.device("cuda", torch.cuda.current_device())
 
     import online_softmax_exact_b200 as osx
-    from online_softmax_exact_b200.schedules import Workspace, ring_attention
+    from online_softmax_exact_b200.schedules import Workspace, ring_attention, ring_slots
     from workloads import attention_inputs
     from workloads.configs import Workload
 
@@ -378,13 +381,15 @@ def run_ours(args, w) -> int:
     P, C = w.n_chunks, w.N // w.n_chunks
     out = (torch.empty((P, B, Hq, C, d), dtype=torch.float32, device=dev),
            torch.empty((P, B, Hq, C), dtype=torch.float32, device=dev))
-    ws = Workspace.for_shape(P * args.streams, B, Hq, C, d, dev)
+    ws = Workspace.for_shape(ring_slots(P, w.causal, args.batched, args.streams), B, Hq, C, d,
+                             dev)
     stream = torch.cuda.current_stream(dev)
     timer = EventTimer(stream)
 
     def step():
         ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
-                       workspace=ws, stream=stream, timer=timer, n_streams=args.streams)
+                       workspace=ws, stream=stream, timer=timer, n_streams=args.streams,
+                       batched=args.batched)
 
     def barrier():
         if world > 1:
@@ -443,7 +448,8 @@ def run_ours(args, w) -> int:
 
     def step1():
         ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
-                       workspace=ws, stream=stream, timer=iso, n_streams=1)
+                       workspace=ws, stream=stream, timer=iso, n_streams=1,
+                       batched=args.batched)
 
     step1()
     torch.cuda.synchronize()
@@ -465,7 +471,8 @@ def run_ours(args, w) -> int:
     # partial buffers, no merge launches
     def step_fused():
         ring_attention(q, k, v, n_chunks=P, causal=w.causal, scale=w.scale, out=out,
-                       stream=stream, n_streams=args.streams, fused_merge=True)
+                       stream=stream, n_streams=args.streams, fused_merge=True,
+                       batched=args.batched)
 
     for _ in range(3):
         step_fused()
@@ -492,7 +499,8 @@ def run_ours(args, w) -> int:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: bf16 N(0,1) from a seeded torch CPU generator",
-        "config": workload_config(w, world, args.streams),
+        "config": workload_config(w, world, None if args.batched else args.streams,
+                                  bool(args.batched)),
         "pct_of_bf16_peak": 100.0 * (value / world) / peak_t,
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128> (attn_fwd_partial)",
                      "achieved": attn_achieved, "peak": peak_t, "unit": "TFLOP/s",
@@ -517,8 +525,8 @@ def run_ours(args, w) -> int:
             "value": w.flops * world / (ms_fused * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms_fused, "steps": n_fused,
             "what": "the same ring step with each query chunk's partials folded into one "
-                    "running (O, LSE) accumulator by attn_fwd_partial_acc: 36 attention "
-                    "launches, no merge launches, no partial buffers"},
+                    "running (O, LSE) accumulator (attn_fwd_partial_acc semantics; batched: "
+                    "one launch per ring step), no merge launches, no partial buffers"},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
@@ -556,7 +564,8 @@ def run_e2e(args, w, q_h, k_h, v_h, dev, out, ws, world) -> dict:
         kd.copy_(kp, non_blocking=True)
         vd.copy_(vp, non_blocking=True)
         ring_attention(qd, kd, vd, n_chunks=w.n_chunks, causal=w.causal, scale=w.scale, out=out,
-                       workspace=ws, stream=stream, n_streams=args.streams)
+                       workspace=ws, stream=stream, n_streams=args.streams,
+                       batched=args.batched)
         o_h.copy_(out[0], non_blocking=True)
         l_h.copy_(out[1], non_blocking=True)
 
@@ -585,7 +594,11 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="ring_32k")
     ap.add_argument("--streams", type=int, default=2,
-                    help="CUDA streams the ring schedule spreads its query chunks over")
+                    help="CUDA streams the ring schedule spreads its query chunks over "
+                         "(per-pair launches only)")
+    ap.add_argument("--batched", type=int, default=1,
+                    help="1: the ring's partials go through attn_fwd_partial_batch "
+                         "(one launch for all pairs); 0: one attn_fwd_partial per pair")
     ap.add_argument("--cpu-seconds", type=float, default=None,
                     help="oracle CPU seconds (baseline sample; per step for --impl reference)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

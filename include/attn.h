@@ -57,6 +57,17 @@ typedef enum {
 } attn_status_t;
 
 #define ATTN_MAX_MERGE_PARTS 64
+#define ATTN_MAX_BATCH_PAIRS 64
+
+/* One (query chunk, key/value chunk) pair of attn_fwd_partial_batch. Rows count in the
+ * parent tensors; o and lse are the pair's own outputs (or accumulators). */
+typedef struct {
+  int64_t q_start, q_len;   /* query rows [q_start, q_start + q_len) */
+  int64_t kv_start, kv_len; /* key/value rows [kv_start, kv_start + kv_len) */
+  int64_t q_off, kv_off;    /* global positions of the first rows (causal test) */
+  float* o;                 /* device, fp32 [B][Hq][q_len][d], 16-byte aligned */
+  float* lse;               /* device, fp32 [B][Hq][q_len], 4-byte aligned */
+} attn_pair_t;
 
 /* Static description of a status code. Never NULL. */
 const char* attn_status_string(int status);
@@ -132,6 +143,24 @@ attn_status_t attn_fwd_partial_acc(const void* q, const void* k_chunk, const voi
                                    int64_t Nq, int64_t Nkv, int64_t q_ld, int64_t kv_ld,
                                    int64_t q_off, int64_t kv_off, int d, int causal,
                                    float scale, void* stream);
+
+/*
+ * attn_fwd_partial_batch - several pairs of attn_fwd_partial (accumulate = 0) or of
+ * attn_fwd_partial_acc (accumulate = 1) over the same parent tensors in ONE launch:
+ * e.g. all the chunk pairs of a ring step, or of a whole emulated ring. Each pair's
+ * result is exactly that of the single-pair call; the work units of all pairs share
+ * one persistent grid, heaviest first, so the tail of one pair is filled by the next.
+ *
+ *   q      device, bf16 parent [B][Hq][q_ld][d];  k, v: parents [B][Hkv][kv_ld][d]
+ *   pairs  HOST array of n_pairs (1 .. ATTN_MAX_BATCH_PAIRS) pair descriptions; every
+ *          chunk must lie inside its parent; no two pairs' outputs may overlap
+ *   other arguments as for attn_fwd_partial. Keys of a parent outside a pair's chunk
+ *   are masked out (never weighted), and must be finite like all inputs.
+ */
+attn_status_t attn_fwd_partial_batch(const void* q, const void* k, const void* v, int B,
+                                     int Hq, int Hkv, int64_t q_ld, int64_t kv_ld, int d,
+                                     int causal, float scale, const attn_pair_t* pairs,
+                                     int n_pairs, int accumulate, void* stream);
 
 /*
  * attn_merge - combine partial results computed over disjoint key sets

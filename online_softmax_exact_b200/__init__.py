@@ -14,6 +14,8 @@ import ctypes
 import torch
 
 from ._abi import (
+    ATTN_MAX_BATCH_PAIRS,
+    AttnPair,
     ATTN_ERR_CUDA,
     ATTN_ERR_INJECTED,
     ATTN_ERR_INVALID_ARG,
@@ -38,7 +40,8 @@ def lib() -> ctypes.CDLL:
 __all__ = [
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA",
     "ATTN_ERR_TIMEOUT", "ATTN_ERR_INJECTED", "ATTN_MAX_MERGE_PARTS", "AttnError",
-    "attn_fwd", "attn_fwd_partial", "attn_fwd_partial_acc", "attn_merge", "attn_device_status", "attn_debug_inject",
+    "attn_fwd", "attn_fwd_partial", "attn_fwd_partial_acc", "attn_fwd_partial_batch",
+    "attn_merge", "ATTN_MAX_BATCH_PAIRS", "attn_device_status", "attn_debug_inject",
     "attn_launch_count", "attn_status_string", "attn_version", "lib",
     "attn_debug_wait_timeout",
 ]
@@ -161,6 +164,39 @@ def attn_fwd_partial_acc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, q
     (o, lse) in place (log-sum-exp merge). Returns (o, lse)."""
     return _partial("attn_fwd_partial_acc", q, k, v, q_start, q_len, kv_start, kv_len,
                     causal, scale, q_off, kv_off, o, lse, stream, alloc=False)
+
+
+def attn_fwd_partial_batch(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pairs, *,
+                           causal: bool, scale: float | None = None, accumulate: bool = False,
+                           stream=None):
+    """Several chunk pairs of the same parents in one launch. ``pairs`` is a sequence of
+    dicts with keys q_start, q_len, kv_start, kv_len, o, lse and optionally q_off, kv_off
+    (default: the row starts). With ``accumulate`` every (o, lse) is an in/out
+    accumulator, as for :func:`attn_fwd_partial_acc`; otherwise it receives the pair's
+    normalised partial."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, Lq, d = q.shape
+    Hkv, Lkv = k.shape[1], k.shape[2]
+    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Hkv, Lkv, d] matching q")
+    if scale is None:
+        scale = d ** -0.5
+    n = len(pairs)
+    arr = (AttnPair * max(n, 1))()
+    for i, pr in enumerate(pairs):
+        o, lse = pr["o"], pr["lse"]
+        _need(o, torch.float32, "o")
+        _need(lse, torch.float32, "lse")
+        if o.shape != (B, Hq, pr["q_len"], d) or lse.shape != (B, Hq, pr["q_len"]):
+            raise ValueError("o / lse must be [B, Hq, q_len, d] / [B, Hq, q_len]")
+        arr[i] = AttnPair(pr["q_start"], pr["q_len"], pr["kv_start"], pr["kv_len"],
+                          pr.get("q_off", pr["q_start"]), pr.get("kv_off", pr["kv_start"]),
+                          o.data_ptr(), lse.data_ptr())
+    st = lib().attn_fwd_partial_batch(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv,
+                                      Lq, Lkv, d, int(bool(causal)), float(scale), arr, n,
+                                      int(bool(accumulate)), _stream_handle(q.device, stream))
+    _check(st, "attn_fwd_partial_batch")
 
 
 def attn_merge(o_parts, lse_parts, *, o: torch.Tensor | None = None,

@@ -17,6 +17,16 @@ ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_INJECTED = 5
 ATTN_MAX_MERGE_PARTS = 64
+ATTN_MAX_BATCH_PAIRS = 64
+
+
+class AttnPair(ctypes.Structure):
+    """attn_pair_t of include/attn.h."""
+
+    _fields_ = [("q_start", ctypes.c_int64), ("q_len", ctypes.c_int64),
+                ("kv_start", ctypes.c_int64), ("kv_len", ctypes.c_int64),
+                ("q_off", ctypes.c_int64), ("kv_off", ctypes.c_int64),
+                ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
 
 STATUS_NAMES = {
     ATTN_OK: "ATTN_OK",
@@ -40,6 +50,9 @@ SIGNATURES = {
     "attn_fwd_partial_acc": (_i32, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                     _i32, _i32, _i32, _i64, _i64, _i64, _i64, _i64, _i64,
                                     _i32, _i32, _f32, _c_void_p]),
+    "attn_fwd_partial_batch": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i64,
+                                      _i64, _i32, _i32, _f32, ctypes.POINTER(AttnPair), _i32,
+                                      _i32, _c_void_p]),
     "attn_merge": (_i32, [ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p), _i32,
                           _c_void_p, _c_void_p, _i64, _i32, _c_void_p]),
     "attn_device_status": (_i32, [_c_void_p, _i32]),

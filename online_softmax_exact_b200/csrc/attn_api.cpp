@@ -69,26 +69,38 @@ attn_status_t check_and_launch(const void* q, const void* k, const void* v, floa
   attn_status_t inj = take_injected();
   if (inj != ATTN_OK) return inj;
 
+  // one pair; the tensor maps cover exactly the two chunks, so rows past a chunk read
+  // as zero
+  osx::PairLaunch pr{0, Nq, 0, Nkv, q_off, kv_off, o, lse};
   osx::FwdLaunch a;
   a.q = q;
   a.k = k;
   a.v = v;
-  a.o = o;
-  a.lse = lse;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
-  a.Nq = Nq;
-  a.Nkv = Nkv;
+  a.q_rows = Nq;
+  a.kv_rows = Nkv;
   a.q_ld = q_ld;
   a.kv_ld = kv_ld;
-  a.q_off = q_off;
-  a.kv_off = kv_off;
   a.d = d;
   a.causal = causal;
   a.scale = scale;
   a.accumulate = accumulate;
+  a.n_pairs = 1;
+  a.pairs = &pr;
   return static_cast<attn_status_t>(osx::launch_fwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+// Cost of a pair's heaviest work unit (its last 256-row block under the causal mask), in
+// key tiles: the batched launch orders pairs by it, heaviest first.
+int64_t pair_heaviest_unit(const attn_pair_t& p, int causal) {
+  const int64_t tiles = (p.kv_len + 127) / 128;
+  if (!causal) return tiles;
+  const int64_t lim = p.q_off + p.q_len - 1 - p.kv_off;
+  if (lim < 0) return 0;
+  const int64_t n = lim / 128 + 1;
+  return n < tiles ? n : tiles;
 }
 
 }  // namespace
@@ -176,6 +188,87 @@ attn_status_t attn_debug_wait_timeout(int64_t limit_cycles, void* stream) {
   if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 31)) return ATTN_ERR_INVALID_ARG;
   return static_cast<attn_status_t>(
       osx::launch_wait_probe(limit_cycles, static_cast<cudaStream_t>(stream)));
+}
+
+attn_status_t attn_fwd_partial_batch(const void* q, const void* k, const void* v, int B, int Hq,
+                                     int Hkv, int64_t q_ld, int64_t kv_ld, int d, int causal,
+                                     float scale, const attn_pair_t* pairs, int n_pairs,
+                                     int accumulate, void* stream) {
+  if (!q || !k || !v || !pairs) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || q_ld < 1 || kv_ld < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return ATTN_ERR_INVALID_ARG;
+  if (n_pairs < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (n_pairs > ATTN_MAX_BATCH_PAIRS) return ATTN_ERR_UNSUPPORTED;
+  if (q_ld > kMaxRows || kv_ld > kMaxRows || (int64_t)B * Hq > (int64_t(1) << 30))
+    return ATTN_ERR_UNSUPPORTED;
+  const uint64_t bh = (uint64_t)B * Hq, bhkv = (uint64_t)B * Hkv;
+  const Span sq = span(q, bh * q_ld * d * 2);
+  const Span sk = span(k, bhkv * kv_ld * d * 2);
+  const Span sv = span(v, bhkv * kv_ld * d * 2);
+  for (int i = 0; i < n_pairs; ++i) {
+    const attn_pair_t& p = pairs[i];
+    if (!p.o || !p.lse || !aligned(p.o, 16) || !aligned(p.lse, 4)) return ATTN_ERR_INVALID_ARG;
+    if (p.q_start < 0 || p.q_len < 1 || p.q_start + p.q_len > q_ld || p.kv_start < 0 ||
+        p.kv_len < 1 || p.kv_start + p.kv_len > kv_ld || p.q_off < 0 || p.kv_off < 0 ||
+        p.q_off > (int64_t(1) << 60) || p.kv_off > (int64_t(1) << 60))
+      return ATTN_ERR_INVALID_ARG;
+    const Span so = span(p.o, bh * p.q_len * d * 4);
+    const Span sl = span(p.lse, bh * p.q_len * 4);
+    if (overlap(so, sq) || overlap(so, sk) || overlap(so, sv) || overlap(sl, sq) ||
+        overlap(sl, sk) || overlap(sl, sv) || overlap(so, sl))
+      return ATTN_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j) {  // no two pairs may write the same memory
+      const Span po = span(pairs[j].o, bh * pairs[j].q_len * d * 4);
+      const Span pl = span(pairs[j].lse, bh * pairs[j].q_len * 4);
+      if (overlap(so, po) || overlap(so, pl) || overlap(sl, po) || overlap(sl, pl))
+        return ATTN_ERR_INVALID_ARG;
+    }
+  }
+  attn_status_t inj = take_injected();
+  if (inj != ATTN_OK) return inj;
+
+  // heaviest pairs first, so that the persistent grid's last units are the light ones
+  int order[ATTN_MAX_BATCH_PAIRS];
+  for (int i = 0; i < n_pairs; ++i) order[i] = i;
+  for (int i = 1; i < n_pairs; ++i) {  // stable insertion sort, n_pairs <= 64
+    const int x = order[i];
+    const int64_t cx = pair_heaviest_unit(pairs[x], causal);
+    int j = i - 1;
+    while (j >= 0 && pair_heaviest_unit(pairs[order[j]], causal) < cx) {
+      order[j + 1] = order[j];
+      --j;
+    }
+    order[j + 1] = x;
+  }
+  osx::PairLaunch pl[ATTN_MAX_BATCH_PAIRS];
+  for (int i = 0; i < n_pairs; ++i) {
+    const attn_pair_t& p = pairs[order[i]];
+    pl[i] = osx::PairLaunch{p.q_start, p.q_len, p.kv_start, p.kv_len, p.q_off, p.kv_off, p.o,
+                            p.lse};
+  }
+  osx::FwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.q_rows = q_ld;
+  a.kv_rows = kv_ld;
+  a.q_ld = q_ld;
+  a.kv_ld = kv_ld;
+  a.d = d;
+  a.causal = causal;
+  a.scale = scale;
+  a.accumulate = accumulate;
+  a.n_pairs = n_pairs;
+  a.pairs = pl;
+  return static_cast<attn_status_t>(osx::launch_fwd(a, static_cast<cudaStream_t>(stream)));
 }
 
 uint64_t attn_launch_count(void) { return osx::launch_count(); }

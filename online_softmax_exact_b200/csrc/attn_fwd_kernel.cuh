@@ -43,21 +43,28 @@
 
 namespace osx {
 
+constexpr int kMaxPairs = 64;
+
+// One (query chunk, key/value chunk) pair of a launch.
+struct PairDesc {
+  float* o;                  // [BH][Nq][D] fp32
+  float* lse;                // [BH][Nq] fp32
+  long long q_off, kv_off;   // global positions of the chunks' first rows (causal test)
+  int q_row0, kv_row0;       // tensor-map row of the chunks' first rows
+  int Nq, Nkv;               // chunk lengths
+};
+
 struct FwdParams {
-  float* o;            // [BH][Nq][D] fp32
-  float* lse;          // [BH][Nq] fp32
   unsigned* status;    // device status word
-  long long Nq, Nkv;   // chunk lengths
-  long long q_off, kv_off;
   int BH;              // B * Hq
   int Hq, Hkv, group;  // group = Hq / Hkv
   int causal;
   float scale_log2;    // scale * log2(e), >= 0
-  int n_qpairs;        // ceil(Nq / 256)
-  int n_units;         // n_qpairs * BH
-  int n_kv_tiles;      // ceil(Nkv / 128)
-  int o_vec8;          // O is 32-byte aligned: store rows with 256-bit stores
+  int o_vec8;          // every O is 32-byte aligned: store rows with 256-bit stores
   int accumulate;      // o/lse hold a partial over other keys: fold this chunk into it
+  int n_pairs;
+  int unit_end[kMaxPairs];  // units of pairs 0..i: sum of ceil(Nq / 256) * BH
+  PairDesc pair[kMaxPairs];
 };
 
 template <int D>
@@ -99,16 +106,41 @@ __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
 
-// Number of key tiles a unit visits: all of them, or under the causal mask those up to
-// the last key visible to the unit's last valid row. 0 means no row sees any key.
-__device__ __forceinline__ int unit_kv_tiles(const FwdParams& p, int qp) {
-  if (!p.causal) return p.n_kv_tiles;
-  long long last_row = (long long)qp * 256 + 255;
-  if (last_row > p.Nq - 1) last_row = p.Nq - 1;
-  const long long lim = p.q_off + last_row - p.kv_off;  // last visible key index
-  if (lim < 0) return 0;
-  const long long n = lim / 128 + 1;
-  return n < p.n_kv_tiles ? (int)n : p.n_kv_tiles;
+// A work unit: 256 query rows (two 128-row tiles) of one (batch, head) of one pair.
+// Units are numbered pair by pair (pairs in launch order, heaviest first), and within a
+// pair from the last row block to the first (heaviest first under the causal mask),
+// heads innermost so that query heads sharing a key/value head run side by side.
+struct Unit {
+  int pair, qp, bh;
+  int n;  // key tiles the unit visits
+};
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+  Unit un;
+  int i = 0;
+  while (i + 1 < p.n_pairs && u >= p.unit_end[i]) ++i;
+  const int ul = u - (i ? p.unit_end[i - 1] : 0);
+  const PairDesc& pr = p.pair[i];
+  const int n_qpairs = (pr.Nq + 255) / 256;
+  const int n_kv_tiles = (pr.Nkv + 127) / 128;
+  un.pair = i;
+  un.qp = n_qpairs - 1 - ul / p.BH;
+  un.bh = ul % p.BH;
+  // all key tiles, or under the causal mask those up to the last key visible to the
+  // unit's last valid row; 0 means no row of the unit sees any key
+  un.n = n_kv_tiles;
+  if (p.causal) {
+    long long last_row = (long long)un.qp * 256 + 255;
+    if (last_row > pr.Nq - 1) last_row = pr.Nq - 1;
+    const long long lim = pr.q_off + last_row - pr.kv_off;  // last visible key index
+    if (lim < 0) {
+      un.n = 0;
+    } else {
+      const long long n = lim / 128 + 1;
+      if (n < n_kv_tiles) un.n = (int)n;
+    }
+  }
+  return un;
 }
 
 // One thread's half row of P for one 128-key tile (64 scores in s): x = S * c - m
@@ -219,6 +251,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int G = gridDim.x;
+  const int n_units = p.unit_end[p.n_pairs - 1];
 
   if (warp >= 16) {
     regs_decrease<C::kRegsOther>();
@@ -229,31 +262,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         bool ok = true;
         for (int r = 0; ok; ++r) {
           const int u = unit_for_round(r, blockIdx.x, G);
-          if (u >= p.n_units) break;
-          const int qp = p.n_qpairs - 1 - u / p.BH;
-          const int bh = u % p.BH;
-          const int n = unit_kv_tiles(p, qp);
+          if (u >= n_units) break;
+          const Unit un = decode_unit(p, u);
+          const int qp = un.qp, bh = un.bh, n = un.n;
           if (n == 0) continue;
+          const PairDesc& pr = p.pair[un.pair];
           const int kvh = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
+          // Q has one shared-memory buffer, so the next unit's Q can only be loaded once
+          // this unit's last Q.K^T has read it; pull it into L2 now so that that load
+          // is short.
+          {
+            const int u2 = unit_for_round(r + 1, blockIdx.x, G);
+            if (u2 < n_units) {
+              const Unit un2 = decode_unit(p, u2);
+              if (un2.n > 0) {
+                const PairDesc& pr2 = p.pair[un2.pair];
+                for (int t = 0; t < 2; ++t)
+                  for (int h = 0; h < D / 64; ++h)
+                    tma_prefetch_l2_3d(&tmQ, h * 64, pr2.q_row0 + un2.qp * 256 + t * 128, un2.bh);
+              }
+            }
+          }
           if (!(ok = mbar_wait(bar(B_QE), (qcount & 1) ^ 1, abort_flag, p.status))) break;
           ++qcount;
           mbar_arrive_expect_tx(bar(B_QF), 2 * C::kTileBytes);
           for (int t = 0; t < 2; ++t)
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + h * 16384, &tmQ, bar(B_QF),
-                          h * 64, qp * 256 + t * 128, bh);
+                          h * 64, pr.q_row0 + qp * 256 + t * 128, bh);
           for (int j = 0; j < n; ++j) {
             if (!(ok = mbar_wait(bar(B_KE + ks), kph ^ 1, abort_flag, p.status))) break;
             mbar_arrive_expect_tx(bar(B_KF + ks), C::kTileBytes);
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sbase + C::kKOff + ks * C::kTileBytes + h * 16384, &tmK, bar(B_KF + ks),
-                          h * 64, j * 128, kvh);
+                          h * 64, pr.kv_row0 + j * 128, kvh);
             if (++ks == C::kStages) { ks = 0; kph ^= 1; }
             if (!(ok = mbar_wait(bar(B_VE + vs), vph ^ 1, abort_flag, p.status))) break;
             mbar_arrive_expect_tx(bar(B_VF + vs), C::kTileBytes);
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sbase + C::kVOff + vs * C::kTileBytes + h * 16384, &tmV, bar(B_VF + vs),
-                          h * 64, j * 128, kvh);
+                          h * 64, pr.kv_row0 + j * 128, kvh);
             if (++vs == C::kStages) { vs = 0; vph ^= 1; }
           }
         }
@@ -298,9 +346,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
         for (int r = 0; ok; ++r) {
           const int u = unit_for_round(r, blockIdx.x, G);
-          if (u >= p.n_units) break;
-          const int qp = p.n_qpairs - 1 - u / p.BH;
-          const int n = unit_kv_tiles(p, qp);
+          if (u >= n_units) break;
+          const int n = decode_unit(p, u).n;
           if (n == 0) continue;
           if (!(ok = mbar_wait(bar(B_QF), qcount & 1, abort_flag, p.status))) break;
           ++qcount;
@@ -377,14 +424,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
     for (int rr = 0; ok; ++rr) {
       const int u = unit_for_round(rr, blockIdx.x, G);
-      if (u >= p.n_units) break;
-      const int qp = p.n_qpairs - 1 - u / p.BH;
-      const int bh = u % p.BH;
-      const int n = unit_kv_tiles(p, qp);
+      if (u >= n_units) break;
+      const Unit un = decode_unit(p, u);
+      const int qp = un.qp, bh = un.bh, n = un.n;
+      const PairDesc& pr = p.pair[un.pair];
       const long long row0 = (long long)qp * 256 + t * 128;  // first row of this tile
       const long long row = row0 + r;
-      const bool row_valid = row < p.Nq;
-      float* orow = p.o + ((long long)bh * p.Nq + row) * D + (D / 2) * h;
+      const bool row_valid = row < pr.Nq;
+      float* orow = pr.o + ((long long)bh * pr.Nq + row) * D + (D / 2) * h;
+      float* lse_row = pr.lse + (long long)bh * pr.Nq + row;
 
       if (n == 0) {
         // no key of this chunk is visible to the unit: the result is empty (O = 0,
@@ -392,16 +440,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (row_valid && !p.accumulate) {
           float4* o4 = reinterpret_cast<float4*>(orow);
           for (int i = 0; i < D / 8; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (h == 0) p.lse[(long long)bh * p.Nq + row] = -INFINITY;
+          if (h == 0) *lse_row = -INFINITY;
         }
         continue;
       }
 
       // last visible key index for this row (local to the chunk), and for the tile's
       // first row (which decides whether a tile needs the per-element mask)
-      long long lim_row = p.Nkv - 1, lim_tile = p.Nkv - 1;
+      long long lim_row = pr.Nkv - 1, lim_tile = pr.Nkv - 1;
       if (p.causal) {
-        const long long a = p.q_off + row - p.kv_off, b = p.q_off + row0 - p.kv_off;
+        const long long a = pr.q_off + row - pr.kv_off, b = pr.q_off + row0 - pr.kv_off;
         lim_row = a < lim_row ? a : lim_row;
         lim_tile = b < lim_tile ? b : lim_tile;
       }
@@ -509,7 +557,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // in accumulate mode both threads of the row read the old LSE before the pair
       // barrier; the new one is written after it
       float lse_acc = -INFINITY;
-      if (p.accumulate && row_valid) lse_acc = p.lse[(long long)bh * p.Nq + row];
+      if (p.accumulate && row_valid) lse_acc = *lse_row;
       *xl_mine = l;
       if (!(ok = pair_sync())) break;
       const float l_row = l + *xl_other;
@@ -572,7 +620,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      if (row_valid && h == 0) p.lse[(long long)bh * p.Nq + row] = lse_out;
+      if (row_valid && h == 0) *lse_row = lse_out;
       tc_fence_before();
     }
     if (!ok) named_bar_arrive(pair_bar, 64);

@@ -7,20 +7,28 @@
 
 namespace osx {
 
-// One attention launch over a (query chunk, key/value chunk) pair; arguments have
-// already been validated by the ABI layer.
+// One (query chunk, key/value chunk) pair of a launch; rows are tensor-map rows.
+struct PairLaunch {
+  long long q_start, q_len, kv_start, kv_len, q_off, kv_off;
+  float* o;
+  float* lse;
+};
+
+// One attention launch over up to kMaxPairs pairs sharing the q/k/v tensor maps;
+// arguments have already been validated by the ABI layer. The maps span q_rows
+// (resp. kv_rows) rows of [B*H][rows][d] views with row strides q_ld / kv_ld.
 struct FwdLaunch {
   const void* q;
   const void* k;
   const void* v;
-  float* o;
-  float* lse;
   int B, Hq, Hkv;
-  long long Nq, Nkv, q_ld, kv_ld, q_off, kv_off;
+  long long q_rows, kv_rows, q_ld, kv_ld;
   int d;
   int causal;
   float scale;
-  int accumulate;  // o/lse are an in/out accumulator (see attn_fwd_partial_acc)
+  int accumulate;  // o/lse are in/out accumulators (see attn_fwd_partial_acc)
+  int n_pairs;
+  const PairLaunch* pairs;
 };
 
 // Returns 0 (ATTN_OK) or an attn_status_t failure code.

@@ -79,32 +79,45 @@ int device_info(DeviceInfo** out) {
 template <int D>
 int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
-  if (!encode_rows_bf16(&tq, a.q, (uint64_t)a.B * a.Hq, a.Nq, a.q_ld, D, 128) ||
-      !encode_rows_bf16(&tk, a.k, (uint64_t)a.B * a.Hkv, a.Nkv, a.kv_ld, D, 128) ||
-      !encode_rows_bf16(&tv, a.v, (uint64_t)a.B * a.Hkv, a.Nkv, a.kv_ld, D, 128))
+  if (!encode_rows_bf16(&tq, a.q, (uint64_t)a.B * a.Hq, a.q_rows, a.q_ld, D, 128) ||
+      !encode_rows_bf16(&tk, a.k, (uint64_t)a.B * a.Hkv, a.kv_rows, a.kv_ld, D, 128) ||
+      !encode_rows_bf16(&tv, a.v, (uint64_t)a.B * a.Hkv, a.kv_rows, a.kv_ld, D, 128))
     return ATTN_ERR_UNSUPPORTED;
+  if (a.n_pairs < 1 || a.n_pairs > kMaxPairs) return ATTN_ERR_UNSUPPORTED;
   FwdParams p;
-  p.o = a.o;
-  p.lse = a.lse;
   p.status = di.status;
-  p.Nq = a.Nq;
-  p.Nkv = a.Nkv;
-  p.q_off = a.q_off;
-  p.kv_off = a.kv_off;
   p.BH = a.B * a.Hq;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.group = a.Hq / a.Hkv;
   p.causal = a.causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
-  p.n_qpairs = static_cast<int>((a.Nq + 255) / 256);
-  const long long units = (long long)p.n_qpairs * p.BH;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  p.n_units = static_cast<int>(units);
-  p.n_kv_tiles = static_cast<int>((a.Nkv + 127) / 128);
-  p.o_vec8 = (reinterpret_cast<uintptr_t>(a.o) % 32) == 0 ? 1 : 0;
   p.accumulate = a.accumulate;
-  const int grid = p.n_units < di.num_sms ? p.n_units : di.num_sms;
+  p.n_pairs = a.n_pairs;
+  p.o_vec8 = 1;
+  long long units = 0;
+  for (int i = 0; i < kMaxPairs; ++i) {
+    PairDesc& d = p.pair[i];
+    if (i >= a.n_pairs) {
+      d = PairDesc{};
+      p.unit_end[i] = static_cast<int>(units);
+      continue;
+    }
+    const PairLaunch& s = a.pairs[i];
+    d.o = s.o;
+    d.lse = s.lse;
+    d.q_off = s.q_off;
+    d.kv_off = s.kv_off;
+    d.q_row0 = static_cast<int>(s.q_start);
+    d.kv_row0 = static_cast<int>(s.kv_start);
+    d.Nq = static_cast<int>(s.q_len);
+    d.Nkv = static_cast<int>(s.kv_len);
+    if ((reinterpret_cast<uintptr_t>(s.o) % 32) != 0) p.o_vec8 = 0;
+    units += ((s.q_len + 255) / 256) * (long long)p.BH;
+    if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    p.unit_end[i] = static_cast<int>(units);
+  }
+  const int grid = units < di.num_sms ? static_cast<int>(units) : di.num_sms;
   attn_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -14,7 +14,7 @@ from dataclasses import dataclass
 
 import torch
 
-from . import attn_fwd_partial, attn_fwd_partial_acc, attn_merge
+from . import attn_fwd_partial, attn_fwd_partial_acc, attn_fwd_partial_batch, attn_merge
 
 
 def chunk_bounds(N: int, n_chunks: int) -> list[tuple[int, int]]:
@@ -112,9 +112,60 @@ class _Streams:
                 t.record_stream(s)
 
 
+def _ring_batched(q, k, v, order, bounds, causal, scale, o_out, l_out, workspace, main,
+                  timer, fused_merge):
+    """The ring schedule with batched launches: without the fused merge, every partial
+    of every query chunk in one launch, then one merge per query chunk; with it, one
+    launch per ring step s holding the step-s pair of every query chunk (so each
+    accumulator is updated once per launch, in ring order)."""
+    P = len(order)
+    if fused_merge:
+        for s_step in range(max(len(x) for x in order)):
+            pairs = []
+            for qi, visit in enumerate(order):
+                if s_step < len(visit):
+                    qs, qe = bounds[qi]
+                    ks, ke = bounds[visit[s_step]]
+                    pairs.append(dict(q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                                      o=o_out[qi], lse=l_out[qi]))
+            with timer("partial", main):
+                attn_fwd_partial_batch(q, k, v, pairs, causal=causal, scale=scale,
+                                       accumulate=s_step > 0, stream=main)
+        return
+    pairs, slots, slot = [], {}, 0
+    for qi, visit in enumerate(order):
+        qs, qe = bounds[qi]
+        for kv in visit:
+            ks, ke = bounds[kv]
+            if len(visit) == 1:
+                o, lse = o_out[qi], l_out[qi]
+            else:
+                o, lse = workspace.o[slot], workspace.lse[slot]
+                slots.setdefault(qi, []).append(slot)
+                slot += 1
+            pairs.append(dict(q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                              o=o, lse=lse))
+    with timer("partial", main):
+        attn_fwd_partial_batch(q, k, v, pairs, causal=causal, scale=scale, stream=main)
+    for qi in range(P):
+        if qi in slots:
+            idx = slots[qi]
+            with timer("merge", main):
+                attn_merge([workspace.o[i] for i in idx], [workspace.lse[i] for i in idx],
+                           o=o_out[qi], lse=l_out[qi], stream=main)
+
+
+def ring_slots(n_chunks: int, causal: bool, batched: bool, n_streams: int = 1) -> int:
+    """Workspace slots (partial buffers) :func:`ring_attention` needs."""
+    order = ring_order(n_chunks, causal)
+    if batched:
+        return sum(len(x) for x in order if len(x) > 1)
+    return max(len(x) for x in order) * max(1, min(n_streams, n_chunks))
+
+
 def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None = None,
                    out=None, workspace: Workspace | None = None, stream=None, timer=None,
-                   n_streams: int = 1, fused_merge: bool = False):
+                   n_streams: int = 1, fused_merge: bool = False, batched: bool = False):
     """Ring Attention's schedule on one GPU: query chunk i attends the key/value chunks
     of :func:`ring_order` one ring step at a time, then merges its partials.
 
@@ -126,7 +177,8 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
     With ``fused_merge`` each query chunk keeps one running (O, LSE) accumulator in the
     output: the first visited chunk writes it, every later ring step folds its partial
     into it (``attn_fwd_partial_acc``), as a ring device does; no partial buffers and
-    no merge launches.
+    no merge launches. With ``batched`` the chunk pairs go through
+    ``attn_fwd_partial_batch`` instead, many pairs per launch (see :func:`_ring_batched`).
     Returns chunk-major (O [P,B,Hq,C,d], LSE [P,B,Hq,C]).
     """
     timer = timer or _NO_TIMER
@@ -135,6 +187,15 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
     C = N // n_chunks
     order = ring_order(n_chunks, causal)
     o_out, l_out = _alloc_out(q, n_chunks, out)
+    if batched:
+        need = ring_slots(n_chunks, causal, True)
+        if not fused_merge and (workspace is None or workspace.o.shape[0] < need
+                                or workspace.o.shape[1:] != (B, Hq, C, d)):
+            workspace = Workspace.for_shape(need, B, Hq, C, d, q.device)
+        main = stream if stream is not None else torch.cuda.current_stream(q.device)
+        _ring_batched(q, k, v, order, bounds, causal, scale, o_out, l_out, workspace, main,
+                      timer, fused_merge)
+        return o_out, l_out
     slots = max(len(x) for x in order)
     n_streams = max(1, min(n_streams, n_chunks))
     need = slots * n_streams

@@ -142,3 +142,28 @@ def test_injection_and_no_device(lib):
     assert fwd(lib) == ATTN_ERR_CUDA
     assert lib.attn_launch_count() == n0
     assert lib.attn_debug_inject(0, 0) == 0
+
+
+def test_batch_argument_checks(lib):
+    from online_softmax_exact_b200._abi import (ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED,
+                                                AttnPair)
+
+    def batch(pairs, n=None, q_ld=1024, kv_ld=1024, d=64, accumulate=0):
+        arr = (AttnPair * max(1, len(pairs)))(*pairs)
+        return lib.attn_fwd_partial_batch(A, 2 * A, 3 * A, 1, 2, 2, q_ld, kv_ld, d, 1, 0.125,
+                                          arr, len(pairs) if n is None else n, accumulate, None)
+
+    big = 1 << 36
+    ok_pair = AttnPair(0, 256, 0, 256, 0, 0, big, big + (1 << 24))
+    assert batch([ok_pair], n=0) == ATTN_ERR_INVALID_ARG
+    assert batch([ok_pair] * 65) == ATTN_ERR_UNSUPPORTED
+    assert batch([ok_pair], d=96) == ATTN_ERR_UNSUPPORTED
+    assert batch([ok_pair], accumulate=2) == ATTN_ERR_INVALID_ARG
+    assert batch([AttnPair(900, 256, 0, 256, 0, 0, big, big + (1 << 24))]) == ATTN_ERR_INVALID_ARG
+    assert batch([AttnPair(0, 256, 0, 0, 0, 0, big, big + (1 << 24))]) == ATTN_ERR_INVALID_ARG
+    assert batch([AttnPair(0, 256, 0, 256, -1, 0, big, big + (1 << 24))]) == ATTN_ERR_INVALID_ARG
+    assert batch([AttnPair(0, 256, 0, 256, 0, 0, None, big)]) == ATTN_ERR_INVALID_ARG
+    assert batch([AttnPair(0, 256, 0, 256, 0, 0, A, big)]) == ATTN_ERR_INVALID_ARG  # o on q
+    # two pairs writing the same output
+    assert batch([ok_pair, AttnPair(256, 256, 0, 256, 0, 0, big, big + (1 << 25))]) == \
+        ATTN_ERR_INVALID_ARG
