@@ -57,7 +57,7 @@ typedef enum {
 } attn_status_t;
 
 #define ATTN_MAX_MERGE_PARTS 64
-#define ATTN_MAX_BATCH_PAIRS 64
+#define ATTN_MAX_BATCH_PAIRS 48
 
 /* One (query chunk, key/value chunk) pair of attn_fwd_partial_batch. Rows count in the
  * parent tensors; o and lse are the pair's own outputs (or accumulators). */

@@ -17,7 +17,7 @@ ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_INJECTED = 5
 ATTN_MAX_MERGE_PARTS = 64
-ATTN_MAX_BATCH_PAIRS = 64
+ATTN_MAX_BATCH_PAIRS = 48
 
 
 class AttnPair(ctypes.Structure):

@@ -43,7 +43,7 @@
 
 namespace osx {
 
-constexpr int kMaxPairs = 64;
+constexpr int kMaxPairs = 48;
 
 // One (query chunk, key/value chunk) pair of a launch.
 struct PairDesc {
@@ -52,6 +52,7 @@ struct PairDesc {
   long long q_off, kv_off;   // global positions of the chunks' first rows (causal test)
   int q_row0, kv_row0;       // tensor-map row of the chunks' first rows
   int Nq, Nkv;               // chunk lengths
+  int uniform;               // every unit visits all key tiles (no causal truncation)
 };
 
 struct FwdParams {
@@ -107,9 +108,11 @@ __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
 }
 
 // A work unit: 256 query rows (two 128-row tiles) of one (batch, head) of one pair.
-// Units are numbered pair by pair (pairs in launch order, heaviest first), and within a
-// pair from the last row block to the first (heaviest first under the causal mask),
-// heads innermost so that query heads sharing a key/value head run side by side.
+// Units are numbered pair by pair (pairs in launch order, heaviest first). Within a pair
+// whose units all cost the same, heads are outermost, so that the CTAs running at one
+// time share the key/value tiles of a few heads in L2; otherwise row blocks go from the
+// last to the first (heaviest first under the causal mask) with heads innermost, query
+// heads sharing a key/value head side by side.
 struct Unit {
   int pair, qp, bh;
   int n;  // key tiles the unit visits
@@ -124,8 +127,13 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   const int n_qpairs = (pr.Nq + 255) / 256;
   const int n_kv_tiles = (pr.Nkv + 127) / 128;
   un.pair = i;
-  un.qp = n_qpairs - 1 - ul / p.BH;
-  un.bh = ul % p.BH;
+  if (pr.uniform) {
+    un.bh = ul / n_qpairs;
+    un.qp = n_qpairs - 1 - ul % n_qpairs;
+  } else {
+    un.qp = n_qpairs - 1 - ul / p.BH;
+    un.bh = ul % p.BH;
+  }
   // all key tiles, or under the causal mask those up to the last key visible to the
   // unit's last valid row; 0 means no row of the unit sees any key
   un.n = n_kv_tiles;

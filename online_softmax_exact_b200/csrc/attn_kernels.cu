@@ -76,6 +76,10 @@ int device_info(DeviceInfo** out) {
   return ATTN_OK;
 }
 
+// three tensor maps plus the parameter block stay within the classic 4 KB of kernel
+// parameters
+static_assert(3 * sizeof(CUtensorMap) + sizeof(FwdParams) <= 4096, "kernel parameters");
+
 template <int D>
 int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
@@ -112,6 +116,13 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
     d.kv_row0 = static_cast<int>(s.kv_start);
     d.Nq = static_cast<int>(s.q_len);
     d.Nkv = static_cast<int>(s.kv_len);
+    {
+      // uniform: even the first row block sees every key tile
+      const long long tiles = (s.kv_len + 127) / 128;
+      const long long last_row0 = (s.q_len < 256 ? s.q_len : 256) - 1;
+      const long long lim0 = s.q_off + last_row0 - s.kv_off;
+      d.uniform = (!a.causal || lim0 >= (tiles - 1) * 128) ? 1 : 0;
+    }
     if ((reinterpret_cast<uintptr_t>(s.o) % 32) != 0) p.o_vec8 = 0;
     units += ((s.q_len + 255) / 256) * (long long)p.BH;
     if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;

@@ -156,7 +156,7 @@ def test_batch_argument_checks(lib):
     big = 1 << 36
     ok_pair = AttnPair(0, 256, 0, 256, 0, 0, big, big + (1 << 24))
     assert batch([ok_pair], n=0) == ATTN_ERR_INVALID_ARG
-    assert batch([ok_pair] * 65) == ATTN_ERR_UNSUPPORTED
+    assert batch([ok_pair] * 49) == ATTN_ERR_UNSUPPORTED
     assert batch([ok_pair], d=96) == ATTN_ERR_UNSUPPORTED
     assert batch([ok_pair], accumulate=2) == ATTN_ERR_INVALID_ARG
     assert batch([AttnPair(900, 256, 0, 256, 0, 0, big, big + (1 << 24))]) == ATTN_ERR_INVALID_ARG
