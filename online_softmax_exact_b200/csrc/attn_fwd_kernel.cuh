@@ -96,10 +96,6 @@ struct FwdCfg {
   static constexpr int kRegsSoftmax = 104;
   static constexpr int kRegsOther = 64;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
-  // In each 16-pair chunk of a half row, pairs i >= kPolyFrom use the FMA-pipe 2^x.
-  // d = 64 needs twice the exponentials per tensor-core FLOP of d = 128, so it hands a
-  // quarter of them to the FMA pipe; at d = 128 the exp unit keeps up on its own.
-  static constexpr int kPolyFrom = (D == 64) ? 12 : 16;
 };
 
 __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
@@ -153,16 +149,15 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
 
 // One thread's half row of P for one 128-key tile (64 scores in s): x = S * c - m
 // (packed pairs), P = 2^x, written to TMEM as 32 columns of bf16 pairs at tP; returns
-// sum(P). Masked tiles send every element through ex2 (so that -inf gives exactly 0).
+// sum(P). Masked elements get x = -inf, for which ex2 gives exactly 0.
 // With kWithMax it also reduces the half-row maximum of the raw scores alongside.
-template <bool kMasked, bool kWithMax, int kPolyFrom>
+template <bool kMasked, bool kWithMax>
 __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP, float c,
                                               float m_use, int climit, float* tile_max) {
   float mx0 = -INFINITY, mx1 = -INFINITY;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  uint64_t A01 = 0, A23 = 0;  // packed partial sums (+0.0f in both halves)
   const uint64_t C2 = f2_pack(c, c);
   const uint64_t NM2 = f2_pack(-m_use, -m_use);
-  const Exp2PolyConsts pk_consts;
 #pragma unroll
   for (int q2 = 0; q2 < 2; ++q2) {
     uint32_t pk[16];
@@ -181,26 +176,21 @@ __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP,
       if (kMasked) {
         if (q2 * 32 + 2 * i > climit) x0 = -INFINITY;
         if (q2 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
-        e0 = ex2_approx(x0);
-        e1 = ex2_approx(x1);
-      } else if (i >= kPolyFrom) {
-        exp2_poly_pair(X, pk_consts, e0, e1);
-      } else {
-        e0 = ex2_approx(x0);
-        e1 = ex2_approx(x1);
       }
-      if (i & 1) {
-        a2 += e0;
-        a3 += e1;
-      } else {
-        a0 += e0;
-        a1 += e1;
-      }
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
+      if (i & 1)
+        A23 = f2_add(A23, f2_pack(e0, e1));
+      else
+        A01 = f2_add(A01, f2_pack(e0, e1));
       pk[i] = pack_bf16x2(e0, e1);
     }
     tmem_st16(tP + q2 * 16, pk);
   }
   if (kWithMax) *tile_max = fmaxf(mx0, mx1);
+  float a0, a1, a2, a3;
+  f2_unpack(A01, a0, a1);
+  f2_unpack(A23, a2, a3);
   return (a0 + a1) + (a2 + a3);
 }
 
@@ -320,7 +310,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
         int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
-        int pcount[2] = {0, 0};
+        int pv_steps = 0;  // P.V steps issued: both tiles' p_full barriers share its parity
         bool ok = true;
         // Descriptors of the stage bases; the descriptor of (address + offset) is the
         // descriptor plus offset >> 4 (the start-address field is the low 14 bits and
@@ -363,16 +353,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int j = 0; j < n && ok; ++j) {
             if (!(ok = mbar_wait(bar(B_KF + ks), kph, abort_flag, p.status))) break;
             tc_fence_after();
+            // (not unrolled: unrolled, the hoisted operand descriptors of both tiles
+            // outgrow this warpgroup's registers)
+#pragma unroll 1
             for (int t = 0; t < 2; ++t) {
               if (j > 0) {
                 if (t == 0) {
                   if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
                 }
-                if (!(ok = mbar_wait(bar(B_PF + t), pcount[t] & 1, abort_flag, p.status))) break;
-                ++pcount[t];
+                if (!(ok = mbar_wait(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
                 tc_fence_after();
                 issue_pv(t, vs, j > 1);
                 if (t == 1) {
+                  ++pv_steps;
                   mma_commit(bar(B_VE + vs));
                   if (++vs == C::kStages) { vs = 0; vph ^= 1; }
                 }
@@ -389,13 +382,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // last P.V of the unit
           if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
           for (int t = 0; t < 2; ++t) {
-            if (!(ok = mbar_wait(bar(B_PF + t), pcount[t] & 1, abort_flag, p.status))) break;
-            ++pcount[t];
+            if (!(ok = mbar_wait(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
             tc_fence_after();
             issue_pv(t, vs, n > 1);
             mma_commit(bar(B_OD + t));
           }
           if (!ok) break;
+          ++pv_steps;
           mma_commit(bar(B_VE + vs));
           if (++vs == C::kStages) { vs = 0; vph ^= 1; }
         }
@@ -439,27 +432,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const long long row0 = (long long)qp * 256 + t * 128;  // first row of this tile
       const long long row = row0 + r;
       const bool row_valid = row < pr.Nq;
-      float* orow = pr.o + ((long long)bh * pr.Nq + row) * D + (D / 2) * h;
-      float* lse_row = pr.lse + (long long)bh * pr.Nq + row;
+      // (the output addresses are formed where they are used, so that they are not
+      // held in registers through the key loop)
+      auto orow_of = [&]() { return pr.o + ((long long)bh * pr.Nq + row) * D + (D / 2) * h; };
+      auto lse_of = [&]() { return pr.lse + (long long)bh * pr.Nq + row; };
 
       if (n == 0) {
         // no key of this chunk is visible to the unit: the result is empty (O = 0,
         // LSE = -inf), and folding an empty result into an accumulator changes nothing
         if (row_valid && !p.accumulate) {
-          float4* o4 = reinterpret_cast<float4*>(orow);
+          float4* o4 = reinterpret_cast<float4*>(orow_of());
           for (int i = 0; i < D / 8; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (h == 0) *lse_row = -INFINITY;
+          if (h == 0) *lse_of() = -INFINITY;
         }
         continue;
       }
 
       // last visible key index for this row (local to the chunk), and for the tile's
       // first row (which decides whether a tile needs the per-element mask)
-      long long lim_row = pr.Nkv - 1, lim_tile = pr.Nkv - 1;
+      // (both in [-1, Nkv - 1], so they fit in int)
+      int lim_row = pr.Nkv - 1, lim_tile = pr.Nkv - 1;
       if (p.causal) {
         const long long a = pr.q_off + row - pr.kv_off, b = pr.q_off + row0 - pr.kv_off;
-        lim_row = a < lim_row ? a : lim_row;
-        lim_tile = b < lim_tile ? b : lim_tile;
+        lim_row = a < lim_row ? (a < -1 ? -1 : (int)a) : lim_row;
+        lim_tile = b < lim_tile ? (b < -1 ? -1 : (int)b) : lim_tile;
       }
 
       float m = -INFINITY;  // running maximum (log2 units) used for the exponent
@@ -479,11 +475,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld_wait(s[0]);
         reg_fence(s[1]);
 
-        const long long kbase = (long long)j * 128 + 64 * h;
-        const bool need_mask = ((long long)j * 128 + 127 > lim_tile);
+        const bool need_mask = (j * 128 + 127 > lim_tile);
         // this half's keys with local column <= climit are visible for this row
-        const long long cl = lim_row - kbase;
-        const int climit = cl < -1 ? -1 : (cl > 63 ? 63 : (int)cl);
+        const int cl = lim_row - (j * 128 + 64 * h);
+        const int climit = cl < -1 ? -1 : (cl > 63 ? 63 : cl);
 
         float m_new, alpha, sum;
         // both warps of a row pair take the same branch (same rows, same m)
@@ -492,7 +487,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // maximum is reduced alongside; the maximum only moves when a row's tile maximum
           // exceeds it by more than 8 (log2 units), and then the warp redoes P.
           float mx;
-          sum = softmax_half<false, true, C::kPolyFrom>(s, tS, c, m, climit, &mx);
+          sum = softmax_half<false, true>(s, tS, c, m, climit, &mx);
           xch_mine[par * 256] = mx;
           if (!(ok = pair_sync())) break;
           mx = fmaxf(mx, xch_other[par * 256]);
@@ -502,7 +497,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           alpha = grow ? ex2_approx(m - m_new) : 1.f;
           if (__any_sync(0xffffffffu, grow)) {
             tmem_st_wait();  // the first P stores land before they are overwritten
-            sum = softmax_half<false, false, C::kPolyFrom>(s, tS, c, m_new, climit, nullptr);
+            sum = softmax_half<false, false>(s, tS, c, m_new, climit, nullptr);
           }
         } else {
           float mx = -INFINITY;
@@ -528,9 +523,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // 1 when unchanged (also when both are -inf), 0 when m was -inf
           alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
           const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          sum = need_mask ? softmax_half<true, false, 16>(s, tS, c, m_use, climit, nullptr)
-                          : softmax_half<false, false, C::kPolyFrom>(s, tS, c, m_use, climit,
-                                                                     nullptr);
+          sum = need_mask ? softmax_half<true, false>(s, tS, c, m_use, climit, nullptr)
+                          : softmax_half<false, false>(s, tS, c, m_use, climit, nullptr);
         }
         l = l * alpha + sum;
 
@@ -565,6 +559,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // in accumulate mode both threads of the row read the old LSE before the pair
       // barrier; the new one is written after it
       float lse_acc = -INFINITY;
+      float* lse_row = lse_of();
       if (p.accumulate && row_valid) lse_acc = *lse_row;
       *xl_mine = l;
       if (!(ok = pair_sync())) break;
@@ -600,7 +595,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld32(tO + q4 * 32, ov);
         tmem_ld_wait(ov);
         if (row_valid) {
-          float* dst = orow + q4 * 32;
+          float* dst = orow_of() + q4 * 32;
           float res[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;

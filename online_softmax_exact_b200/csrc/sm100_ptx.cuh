@@ -1,6 +1,6 @@
 // sm100_ptx.cuh - thin inline-PTX wrappers for the sm_100a features the kernels use:
 // mbarriers with bounded waits, TMA tiled loads, the tcgen05 tensor-core / tensor
-// memory (TMEM) instructions, packed fp32 pairs, and a polynomial 2^x on the FMA pipe.
+// memory (TMEM) instructions and packed fp32 pairs.
 #pragma once
 
 #include <cstdint>
@@ -298,12 +298,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return d;
 }
 
-// Coefficients of p(f) ~ 2^f on [-1/2, 1/2], p(f) = 1 + c1 f + c2 f^2 + c3 f^3, fitted by
-// exp2_poly_fit.py (max relative error 1.03e-4 evaluated in fp32).
-constexpr float kExp2C1 = 6.932863593e-01f;
-constexpr float kExp2C2 = 2.422038764e-01f;
-constexpr float kExp2C3 = 5.498712510e-02f;
-
 // 256-bit global store of 8 floats (address 32-byte aligned)
 __device__ __forceinline__ void st_global_v8(float* p, float a0, float a1, float a2, float a3,
                                              float a4, float a5, float a6, float a7) {
@@ -337,45 +331,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// 2^x for a pair of finite x <= 64 on the FMA pipe: x clamped below at -125, n =
-// round(x) by the 1.5*2^23 shifter, f = x - n in [-1/2, 1/2], 2^f by a degree-3
-// polynomial (coefficients fitted by exp2_poly_fit.py for minimum relative error:
-// 1.03e-4 at most), and n added to the exponent field. Inputs below -125 give 2^-125
-// or so instead of a smaller value; callers only pass rows whose denominator is >= 1.
-// The pair stays packed (f32x2 arithmetic) from the input to the exponent add.
-struct Exp2PolyConsts {
-  uint64_t shift, c3, c2, c1, one;
-  __device__ __forceinline__ Exp2PolyConsts()
-      : shift(f2_pack(12582912.0f, 12582912.0f)),  // 1.5 * 2^23
-        c3(f2_pack(kExp2C3, kExp2C3)),
-        c2(f2_pack(kExp2C2, kExp2C2)),
-        c1(f2_pack(kExp2C1, kExp2C1)),
-        one(f2_pack(1.0f, 1.0f)) {}
-};
-
-__device__ __forceinline__ void exp2_poly_pair(uint64_t X, const Exp2PolyConsts& k, float& y0,
-                                               float& y1) {
-  float x0, x1;
-  f2_unpack(X, x0, x1);
-  const uint64_t Xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t J = f2_add(Xc, k.shift);           // shift + round(x): n in the low bits
-  const uint64_t F = f2_sub(Xc, f2_sub(J, k.shift));  // f = x - round(x) in [-1/2, 1/2]
-  uint64_t P = f2_fma(k.c3, F, k.c2);
-  P = f2_fma(P, F, k.c1);
-  P = f2_fma(P, F, k.one);
-  uint32_t p0, p1, j0, j1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(P));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(J));
-  // (shift + n) << 23 leaves exactly n << 23 in 32 bits
-  y0 = __uint_as_float(j0 * 8388608u + p0);
-  y1 = __uint_as_float(j1 * 8388608u + p1);
 }
 
 }  // namespace osx
