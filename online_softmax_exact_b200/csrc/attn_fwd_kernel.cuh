@@ -323,18 +323,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // O_t += P_t V (stage vstage); acc=false overwrites O_t. P_t's keys 0-63 sit in
         // S_t columns [0,32), keys 64-127 in [64,96).
         auto issue_pv = [&](int t, int vstage, bool acc) {
-          const uint64_t dv = dv0 + (uint64_t)vstage * kTileStep;
+          uint64_t dv = dv0 + (uint64_t)vstage * kTileStep;
           const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0);
           const uint32_t tP = tmem + (t ? C::kColS1 : C::kColS0);
+          opaque(dv);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tO, tP + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), dv + (uint64_t)(kk * 128),
                    idesc_pv, (acc || kk > 0) ? 1u : 0u);
         };
         auto issue_qk = [&](int t, int kstage) {
-          const uint64_t dq = dq0 + (uint64_t)t * kTileStep;
-          const uint64_t dk = dk0 + (uint64_t)kstage * kTileStep;
+          uint64_t dq = dq0 + (uint64_t)t * kTileStep;
+          uint64_t dk = dk0 + (uint64_t)kstage * kTileStep;
           const uint32_t tS = tmem + (t ? C::kColS1 : C::kColS0);
+          opaque(dq);
+          opaque(dk);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)((kk / 4) * 1024 + (kk % 4) * 2);
@@ -353,9 +356,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int j = 0; j < n && ok; ++j) {
             if (!(ok = mbar_wait(bar(B_KF + ks), kph, abort_flag, p.status))) break;
             tc_fence_after();
-            // (not unrolled: unrolled, the hoisted operand descriptors of both tiles
-            // outgrow this warpgroup's registers)
-#pragma unroll 1
             for (int t = 0; t < 2; ++t) {
               if (j > 0) {
                 if (t == 0) {

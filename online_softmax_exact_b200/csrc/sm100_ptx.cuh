@@ -313,6 +313,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Hides a value's origin from the optimiser, so that expressions derived from it are
+// formed where they are used rather than hoisted out of loops (and held in registers).
+__device__ __forceinline__ void opaque(uint64_t& v) { asm volatile("" : "+l"(v)); }
+
 // packed fp32 pairs (sm_100): {lo, hi} in one 64-bit register pair
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t d;
