@@ -28,6 +28,7 @@ problem of the same size (different seed): weak scaling, no data-path collective
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -92,6 +93,28 @@ def load_peaks() -> tuple[dict, str]:
         except Exception:
             pass
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of ONE attention launch of
+# the default step, from one ncu capture of `bench.py --steps 3 --warmup 3
+# --no-cpu-baseline` (summarised with its command under profiles/). Keyed by the
+# digest of the kernel sources the capture ran, and by launch mode; any other source
+# gives null.
+MEASURED_TRAFFIC: dict[str, dict[str, float]] = {}
+
+
+def kernel_source_digest() -> str:
+    """SHA-256 over the attention kernel's device sources (the files whose change
+    invalidates a DRAM-traffic capture)."""
+    h = hashlib.sha256()
+    for name in ("attn_fwd_kernel.cuh", "sm100_ptx.cuh"):
+        h.update((ROOT / "online_softmax_exact_b200" / "csrc" / name).read_bytes())
+    return h.hexdigest()
+
+
+def measured_traffic(batched: bool) -> float | None:
+    return MEASURED_TRAFFIC.get(kernel_source_digest(), {}).get(
+        "batched" if batched else "per_pair")
 
 
 def ring_step_plan(n_chunks: int, causal: bool):
@@ -502,12 +525,17 @@ def run_ours(args, w) -> int:
         "config": workload_config(w, world, None if args.batched else args.streams,
                                   bool(args.batched)),
         "pct_of_bf16_peak": 100.0 * (value / world) / peak_t,
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128> (attn_fwd_partial)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_fwd_kernel<128> (" + ("attn_fwd_partial_batch"
+                                                           if args.batched else
+                                                           "attn_fwd_partial") + ")",
                      "achieved": attn_achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attn_achieved / peak_t,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a "
                                     f"long back-to-back loop)",
-                     "traffic": None,
+                     "traffic": measured_traffic(bool(args.batched)),
+                     "traffic_note": "DRAM bytes per attention launch from one ncu capture "
+                                     "of this kernel source; null if the source changed",
                      "launches": n_part, "busy_ms": t_part, "summed_launch_ms": sum_part,
                      "timing": "achieved = algorithmic FLOPs of all attention launches in the "
                                "timed region / the device time during which at least one was "

@@ -132,3 +132,13 @@ def test_event_timer_busy_time_is_the_union_of_intervals():
     tot = t.totals(Ev(0))
     assert tot["partial"] == (4.0, 3, 5.0)      # [0,3] and [5,6]
     assert tot["merge"] == (1.0, 1, 1.0)
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel_source(monkeypatch):
+    digest = bench.kernel_source_digest()
+    assert len(digest) == 64
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {digest: {"batched": 7.0e9}})
+    assert bench.measured_traffic(True) == 7.0e9
+    assert bench.measured_traffic(False) is None
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {"0" * 64: {"batched": 7.0e9}})
+    assert bench.measured_traffic(True) is None
