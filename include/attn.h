@@ -185,6 +185,45 @@ attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_pa
                          void* stream);
 
 /*
+ * attn_ring_fwd_host - Ring Attention's schedule on one GPU, from HOST buffers to
+ * HOST buffers ("Ring Attention with Blockwise Parallel Transformers", section 3:
+ * the sequence is cut into blocks; at ring step s the holder of query block i
+ * attends key/value block (i - s) mod n_chunks, and its partial results are
+ * combined). The sequence is cut into n_chunks chunks of C = N / n_chunks rows;
+ * query chunk i attends, in ring order, every key/value chunk (under the causal
+ * mask only chunks 0..i), one attn_fwd_partial_batch launch per query chunk, and
+ * its partials are combined with attn_merge. Results equal those of the same
+ * calls made one by one on device buffers.
+ *
+ * The copies are pipelined with the compute: each chunk of q, k, v goes to the
+ * device on h2d_stream as a strided copy, query chunk i's launch waits only for
+ * the chunks it reads, and its merged result goes back on d2h_stream as soon as
+ * it is final. The call is asynchronous like the others; the work is ordered after
+ * earlier work on `stream`, and later work on `stream` waits for all of it,
+ * including the last copy back.
+ *
+ *   q_h, k_h, v_h   HOST, bf16 [B][Hq][N][d], [B][Hkv][N][d]; page-locked memory
+ *                   lets the copies overlap (pageable memory works, unoverlapped)
+ *   o_h, lse_h      HOST, fp32 chunk-major [n_chunks][B][Hq][C][d] and
+ *                   [n_chunks][B][Hq][C] (written)
+ *   q_d, k_d, v_d   DEVICE staging, same shapes as q_h, k_h, v_h (16-byte aligned)
+ *   o_d, lse_d      DEVICE, same shapes as o_h, lse_h (o_d 32-byte aligned)
+ *   ws_o, ws_lse    DEVICE partial buffers, ws_slots slots of [B][Hq][C][d] and
+ *                   [B][Hq][C] (ws_o 32-byte aligned); ws_slots must be at least
+ *                   the number of chunks a query chunk visits when that is more than
+ *                   one (n_chunks), else 0 and the pointers may be NULL
+ *   n_chunks        1 .. ATTN_MAX_BATCH_PAIRS, dividing N
+ *   h2d_stream, d2h_stream  streams for the two copy directions (NULL: `stream`)
+ *   other arguments as for attn_fwd. Device buffers must not overlap each other.
+ */
+attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v_h,
+                                 float* o_h, float* lse_h, void* q_d, void* k_d, void* v_d,
+                                 float* o_d, float* lse_d, float* ws_o, float* ws_lse,
+                                 int ws_slots, int B, int Hq, int Hkv, int64_t N, int d,
+                                 int n_chunks, int causal, float scale, void* stream,
+                                 void* h2d_stream, void* d2h_stream);
+
+/*
  * attn_device_status - synchronise `stream` and report whether any kernel of this
  * library on the current device recorded a device-side failure since the last
  * reset (ATTN_ERR_TIMEOUT: a bounded wait ran out; the kernel then stopped its
@@ -195,7 +234,7 @@ attn_status_t attn_device_status(void* stream, int reset);
 
 /*
  * attn_debug_inject - host-side fault injection for tests of error paths: the next
- * `count` calls of attn_fwd, attn_fwd_partial or attn_merge return `status`
+ * `count` calls of an entry point that launches work return `status`
  * (which must be a failure code) after argument checks and before any launch.
  * count = 0 disarms. Not thread-safe; for tests only.
  */

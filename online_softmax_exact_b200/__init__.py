@@ -43,7 +43,7 @@ __all__ = [
     "attn_fwd", "attn_fwd_partial", "attn_fwd_partial_acc", "attn_fwd_partial_batch",
     "attn_merge", "ATTN_MAX_BATCH_PAIRS", "attn_device_status", "attn_debug_inject",
     "attn_launch_count", "attn_status_string", "attn_version", "lib",
-    "attn_debug_wait_timeout",
+    "attn_debug_wait_timeout", "attn_ring_fwd_host", "RingHostBuffers",
 ]
 
 
@@ -229,6 +229,99 @@ def attn_merge(o_parts, lse_parts, *, o: torch.Tensor | None = None,
                          _stream_handle(ref.device, stream))
     _check(st, "attn_merge")
     return o, lse
+
+
+class RingHostBuffers:
+    """Device buffers of :func:`attn_ring_fwd_host`: bf16 staging for q, k, v
+    ([B, H, N, d]), the chunk-major fp32 result (O [P, B, Hq, C, d], LSE [P, B, Hq, C])
+    and the partial slots (P of them when P > 1)."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, N: int, d: int, n_chunks: int, device):
+        if n_chunks < 1 or N % n_chunks:
+            raise ValueError("the sequence length must split into equal chunks")
+        C = N // n_chunks
+        bf = dict(dtype=torch.bfloat16, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.shape = (B, Hq, Hkv, N, d, n_chunks)
+        self.q = torch.empty((B, Hq, N, d), **bf)
+        self.k = torch.empty((B, Hkv, N, d), **bf)
+        self.v = torch.empty((B, Hkv, N, d), **bf)
+        self.o = torch.empty((n_chunks, B, Hq, C, d), **f32)
+        self.lse = torch.empty((n_chunks, B, Hq, C), **f32)
+        slots = n_chunks if n_chunks > 1 else 0
+        self.ws_o = torch.empty((max(slots, 1), B, Hq, C, d), **f32)
+        self.ws_lse = torch.empty((max(slots, 1), B, Hq, C), **f32)
+        self.slots = slots
+
+    def tensors(self):
+        return [self.q, self.k, self.v, self.o, self.lse, self.ws_o, self.ws_lse]
+
+
+_copy_streams: dict = {}
+
+
+def _host_copy_streams(device: torch.device):
+    if device.index not in _copy_streams:
+        _copy_streams[device.index] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    return _copy_streams[device.index]
+
+
+def attn_ring_fwd_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, *,
+                       n_chunks: int, causal: bool, scale: float | None = None,
+                       o_h: torch.Tensor | None = None, lse_h: torch.Tensor | None = None,
+                       buffers: RingHostBuffers | None = None, device=None, stream=None,
+                       h2d_stream=None, d2h_stream=None):
+    """Ring Attention's schedule on one GPU from host tensors to host tensors, with the
+    copies pipelined against the compute (see attn_ring_fwd_host in attn.h).
+    q_h / k_h / v_h: CPU bf16 [B, H, N, d] (page-locked for overlap). Returns the
+    chunk-major CPU fp32 (O [P, B, Hq, C, d], LSE [P, B, Hq, C]); the copies are
+    asynchronous, so synchronise ``stream`` before reading them."""
+    for t, n in ((q_h, "q_h"), (k_h, "k_h"), (v_h, "v_h")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 \
+                or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CPU bf16 tensor")
+    B, Hq, N, d = q_h.shape
+    Hkv = k_h.shape[1]
+    if v_h.shape != k_h.shape or k_h.shape[0] != B or k_h.shape[2] != N or k_h.shape[3] != d:
+        raise ValueError("k_h and v_h must be [B, Hkv, N, d] matching q_h")
+    if n_chunks < 1 or N % n_chunks:
+        raise ValueError("the sequence length must split into equal chunks")
+    C = N // n_chunks
+    dev = torch.device(device) if device is not None else \
+        torch.device("cuda", torch.cuda.current_device())
+    if buffers is None:
+        buffers = RingHostBuffers(B, Hq, Hkv, N, d, n_chunks, dev)
+    elif buffers.shape != (B, Hq, Hkv, N, d, n_chunks):
+        raise ValueError("buffers were made for another shape")
+    if o_h is None:
+        o_h = torch.empty((n_chunks, B, Hq, C, d), dtype=torch.float32).pin_memory()
+    if lse_h is None:
+        lse_h = torch.empty((n_chunks, B, Hq, C), dtype=torch.float32).pin_memory()
+    for t, shape, n in ((o_h, (n_chunks, B, Hq, C, d), "o_h"),
+                        (lse_h, (n_chunks, B, Hq, C), "lse_h")):
+        if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() \
+                or tuple(t.shape) != shape:
+            raise ValueError(f"{n} must be a contiguous CPU fp32 tensor of shape {shape}")
+    if scale is None:
+        scale = d ** -0.5
+    s_main = stream if stream is not None else torch.cuda.current_stream(dev)
+    if h2d_stream is None or d2h_stream is None:
+        hs, ds = _host_copy_streams(dev)
+        h2d_stream = h2d_stream or hs
+        d2h_stream = d2h_stream or ds
+    for t in buffers.tensors():  # also used on the copy streams
+        t.record_stream(h2d_stream)
+        t.record_stream(d2h_stream)
+    b = buffers
+    st = lib().attn_ring_fwd_host(
+        q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
+        b.q.data_ptr(), b.k.data_ptr(), b.v.data_ptr(), b.o.data_ptr(), b.lse.data_ptr(),
+        b.ws_o.data_ptr() if b.slots else None, b.ws_lse.data_ptr() if b.slots else None,
+        b.slots, B, Hq, Hkv, N, d, n_chunks, int(bool(causal)), float(scale),
+        _stream_handle(dev, s_main), _stream_handle(dev, h2d_stream),
+        _stream_handle(dev, d2h_stream))
+    _check(st, "attn_ring_fwd_host")
+    return o_h, lse_h
 
 
 def attn_device_status(stream=None, reset: bool = False) -> int:

@@ -55,6 +55,9 @@ SIGNATURES = {
                                       _i32, _c_void_p]),
     "attn_merge": (_i32, [ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p), _i32,
                           _c_void_p, _c_void_p, _i64, _i32, _c_void_p]),
+    "attn_ring_fwd_host": (_i32, [_c_void_p] * 12 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32,
+                                                     _i32, _f32, _c_void_p, _c_void_p,
+                                                     _c_void_p]),
     "attn_device_status": (_i32, [_c_void_p, _i32]),
     "attn_debug_inject": (_i32, [_i32, _i32]),
     "attn_debug_wait_timeout": (_i32, [_i64, _c_void_p]),

@@ -3,6 +3,7 @@
 // arguments are reported without touching a device.
 #include <cmath>
 #include <cstdint>
+#include <vector>
 
 #include "../../include/attn.h"
 #include "attn_internal.h"
@@ -235,7 +236,7 @@ attn_status_t attn_fwd_partial_batch(const void* q, const void* k, const void* v
   // heaviest pairs first, so that the persistent grid's last units are the light ones
   int order[ATTN_MAX_BATCH_PAIRS];
   for (int i = 0; i < n_pairs; ++i) order[i] = i;
-  for (int i = 1; i < n_pairs; ++i) {  // stable insertion sort, n_pairs <= 64
+  for (int i = 1; i < n_pairs; ++i) {  // stable insertion sort, n_pairs <= 48
     const int x = order[i];
     const int64_t cx = pair_heaviest_unit(pairs[x], causal);
     int j = i - 1;
@@ -269,6 +270,130 @@ attn_status_t attn_fwd_partial_batch(const void* q, const void* k, const void* v
   a.n_pairs = n_pairs;
   a.pairs = pl;
   return static_cast<attn_status_t>(osx::launch_fwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v_h, float* o_h,
+                                 float* lse_h, void* q_d, void* k_d, void* v_d, float* o_d,
+                                 float* lse_d, float* ws_o, float* ws_lse, int ws_slots, int B,
+                                 int Hq, int Hkv, int64_t N, int d, int n_chunks, int causal,
+                                 float scale, void* stream, void* h2d_stream, void* d2h_stream) {
+  if (!q_h || !k_h || !v_h || !o_h || !lse_h || !q_d || !k_d || !v_d || !o_d || !lse_d)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || N < 1) return ATTN_ERR_INVALID_ARG;
+  if (n_chunks < 1 || N % n_chunks != 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q_d, 16) || !aligned(k_d, 16) || !aligned(v_d, 16) || !aligned(o_d, 32) ||
+      !aligned(lse_d, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (n_chunks > ATTN_MAX_BATCH_PAIRS) return ATTN_ERR_UNSUPPORTED;
+  if (N > kMaxRows || (int64_t)B * Hq > (int64_t(1) << 30)) return ATTN_ERR_UNSUPPORTED;
+  // the last query chunk visits every key/value chunk (causal or not)
+  const int need = n_chunks > 1 ? n_chunks : 0;
+  if (ws_slots < need) return ATTN_ERR_INVALID_ARG;
+  if (need > 0 && (!ws_o || !ws_lse || !aligned(ws_o, 32) || !aligned(ws_lse, 4)))
+    return ATTN_ERR_INVALID_ARG;
+  const int64_t C = N / n_chunks;
+  const uint64_t bh = (uint64_t)B * Hq, bhkv = (uint64_t)B * Hkv;
+  const uint64_t slot_rows = bh * (uint64_t)C;
+  std::vector<Span> dev = {span(q_d, bh * N * d * 2), span(k_d, bhkv * N * d * 2),
+                           span(v_d, bhkv * N * d * 2), span(o_d, bh * N * d * 4),
+                           span(lse_d, bh * N * 4)};
+  if (need > 0) {
+    dev.push_back(span(ws_o, need * slot_rows * d * 4));
+    dev.push_back(span(ws_lse, need * slot_rows * 4));
+  }
+  for (size_t i = 0; i < dev.size(); ++i)
+    for (size_t j = 0; j < i; ++j)
+      if (overlap(dev[i], dev[j])) return ATTN_ERR_INVALID_ARG;
+  attn_status_t inj = take_injected();
+  if (inj != ATTN_OK) return inj;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t sh = h2d_stream ? static_cast<cudaStream_t>(h2d_stream) : s;
+  cudaStream_t sd = d2h_stream ? static_cast<cudaStream_t>(d2h_stream) : s;
+  // events: [0] start, [1] end, [2 + c] chunk c on the device, [2 + P + i] result i final
+  std::vector<cudaEvent_t> ev(2 + 2 * (size_t)n_chunks, nullptr);
+  auto release = [&]() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);  // resources are released once pending work completes
+  };
+  for (auto& e : ev) {
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      e = nullptr;
+      release();
+      return ATTN_ERR_CUDA;
+    }
+  }
+  attn_status_t st = ATTN_OK;
+  auto cuda_ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
+    return st == ATTN_OK;
+  };
+  auto after = [&](cudaStream_t waiter, cudaEvent_t e, cudaStream_t signaller) {
+    if (waiter == signaller) return true;  // stream order already covers it
+    return cuda_ok(cudaEventRecord(e, signaller)) && cuda_ok(cudaStreamWaitEvent(waiter, e, 0));
+  };
+  // the copies in overwrite the staging buffers: after earlier work on `stream`
+  // (the copies back wait for events recorded on `stream`, so they follow it anyway)
+  after(sh, ev[0], s);
+
+  // host -> device: chunk c of k, v, q as strided copies (B*H runs of C rows)
+  const size_t pitch = (size_t)N * d * 2, width = (size_t)C * d * 2;
+  for (int c = 0; c < n_chunks && st == ATTN_OK; ++c) {
+    const size_t off = (size_t)c * width;
+    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(k_d) + off, pitch,
+                              static_cast<const char*>(k_h) + off, pitch, width, bhkv,
+                              cudaMemcpyHostToDevice, sh));
+    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(v_d) + off, pitch,
+                              static_cast<const char*>(v_h) + off, pitch, width, bhkv,
+                              cudaMemcpyHostToDevice, sh));
+    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(q_d) + off, pitch,
+                              static_cast<const char*>(q_h) + off, pitch, width, bh,
+                              cudaMemcpyHostToDevice, sh));
+    if (st == ATTN_OK && sh != s) cuda_ok(cudaEventRecord(ev[2 + c], sh));
+  }
+
+  // per query chunk: its partials in one launch, their merge, and the copy back
+  attn_pair_t pairs[ATTN_MAX_BATCH_PAIRS];
+  const float* po[ATTN_MAX_BATCH_PAIRS];
+  const float* pl[ATTN_MAX_BATCH_PAIRS];
+  for (int qi = 0; qi < n_chunks && st == ATTN_OK; ++qi) {
+    if (sh != s && !cuda_ok(cudaStreamWaitEvent(s, ev[2 + (causal ? qi : n_chunks - 1)], 0)))
+      break;
+    float* o_i = o_d + (size_t)qi * slot_rows * d;
+    float* l_i = lse_d + (size_t)qi * slot_rows;
+    int nv = 0;
+    for (int step = 0; step < n_chunks; ++step) {
+      const int kv = ((qi - step) % n_chunks + n_chunks) % n_chunks;
+      if (causal && kv > qi) continue;
+      pairs[nv] = attn_pair_t{qi * C, C, kv * C, C, qi * C, kv * C, nullptr, nullptr};
+      ++nv;
+    }
+    for (int j = 0; j < nv; ++j) {
+      pairs[j].o = nv == 1 ? o_i : ws_o + (size_t)j * slot_rows * d;
+      pairs[j].lse = nv == 1 ? l_i : ws_lse + (size_t)j * slot_rows;
+      po[j] = pairs[j].o;
+      pl[j] = pairs[j].lse;
+    }
+    st = attn_fwd_partial_batch(q_d, k_d, v_d, B, Hq, Hkv, N, N, d, causal, scale, pairs, nv, 0,
+                                stream);
+    if (st == ATTN_OK && nv > 1)
+      st = attn_merge(po, pl, nv, o_i, l_i, (int64_t)slot_rows, d, stream);
+    if (st != ATTN_OK) break;
+    if (sd != s && !(cuda_ok(cudaEventRecord(ev[2 + n_chunks + qi], s)) &&
+                     cuda_ok(cudaStreamWaitEvent(sd, ev[2 + n_chunks + qi], 0))))
+      break;
+    cuda_ok(cudaMemcpyAsync(o_h + (size_t)qi * slot_rows * d, o_i, slot_rows * d * 4,
+                            cudaMemcpyDeviceToHost, sd));
+    cuda_ok(cudaMemcpyAsync(lse_h + (size_t)qi * slot_rows, l_i, slot_rows * 4,
+                            cudaMemcpyDeviceToHost, sd));
+  }
+  // later work on `stream` waits for the last copy back
+  if (st == ATTN_OK) after(s, ev[1], sd);
+  release();
+  return st;
 }
 
 uint64_t attn_launch_count(void) { return osx::launch_count(); }

@@ -167,3 +167,45 @@ def test_batch_argument_checks(lib):
     # two pairs writing the same output
     assert batch([ok_pair, AttnPair(256, 256, 0, 256, 0, 0, big, big + (1 << 25))]) == \
         ATTN_ERR_INVALID_ARG
+
+
+def test_ring_host_argument_checks(lib):
+    """attn_ring_fwd_host checks every argument before any CUDA call; with no device a
+    valid call fails only at the first CUDA call, and an injected failure before it."""
+    import torch
+
+    from online_softmax_exact_b200._abi import (ATTN_ERR_CUDA, ATTN_ERR_INJECTED,
+                                                ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED)
+
+    G = 1 << 32  # device buffers 4 GiB apart (B=1, H=2, N=1024, d=64 needs far less)
+    H = 1 << 44  # fake host addresses, never dereferenced by the checks
+
+    def ring(q_h=H, k_h=H + A, v_h=H + 2 * A, o_h=H + 3 * A, lse_h=H + 4 * A, q_d=G,
+             k_d=2 * G, v_d=3 * G, o_d=4 * G, lse_d=5 * G, ws_o=6 * G, ws_lse=7 * G,
+             ws_slots=4, B=1, Hq=2, Hkv=2, N=1024, d=64, n_chunks=4, causal=1, scale=0.125):
+        return lib.attn_ring_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,
+                                      ws_o, ws_lse, ws_slots, B, Hq, Hkv, N, d, n_chunks, causal,
+                                      scale, None, None, None)
+
+    assert ring(q_h=None) == ATTN_ERR_INVALID_ARG
+    assert ring(lse_d=None) == ATTN_ERR_INVALID_ARG
+    assert ring(n_chunks=3) == ATTN_ERR_INVALID_ARG            # 1024 rows do not split in 3
+    assert ring(n_chunks=0) == ATTN_ERR_INVALID_ARG
+    assert ring(n_chunks=64, N=64 * 16) == ATTN_ERR_UNSUPPORTED
+    assert ring(d=96) == ATTN_ERR_UNSUPPORTED
+    assert ring(causal=2) == ATTN_ERR_INVALID_ARG
+    assert ring(scale=float("nan")) == ATTN_ERR_INVALID_ARG
+    assert ring(o_d=4 * G + 16) == ATTN_ERR_INVALID_ARG         # merge output needs 32 bytes
+    assert ring(ws_slots=3) == ATTN_ERR_INVALID_ARG             # the last chunk visits 4
+    assert ring(ws_o=None) == ATTN_ERR_INVALID_ARG
+    assert ring(ws_lse=5 * G) == ATTN_ERR_INVALID_ARG           # overlaps lse_d
+    assert ring(k_d=G + 4096) == ATTN_ERR_INVALID_ARG           # overlaps q_d
+    assert ring(Hq=3, Hkv=2) == ATTN_ERR_INVALID_ARG
+    if torch.cuda.is_available():
+        return
+    # one chunk needs no partial buffers
+    assert lib.attn_debug_inject(ATTN_ERR_INJECTED, 1) == 0
+    assert ring(n_chunks=1, ws_o=None, ws_lse=None, ws_slots=0) == ATTN_ERR_INJECTED
+    n0 = lib.attn_launch_count()
+    assert ring() == ATTN_ERR_CUDA
+    assert lib.attn_launch_count() == n0
