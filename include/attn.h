@@ -191,15 +191,16 @@ attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_pa
  * attends key/value block (i - s) mod n_chunks, and its partial results are
  * combined). The sequence is cut into n_chunks chunks of C = N / n_chunks rows;
  * query chunk i attends, in ring order, every key/value chunk (under the causal
- * mask only chunks 0..i), one attn_fwd_partial_batch launch per query chunk, and
- * its partials are combined with attn_merge. Results equal those of the same
- * calls made one by one on device buffers.
+ * mask only chunks 0..i); each pair is one partial (attn_fwd_partial_batch
+ * launches) and a query chunk's partials are combined in ring order with
+ * attn_merge. Results equal those of the same calls made on device buffers.
  *
- * The copies are pipelined with the compute: each chunk of q, k, v goes to the
- * device on h2d_stream as a strided copy, query chunk i's launch waits only for
- * the chunks it reads, and its merged result goes back on d2h_stream as soon as
- * it is final. The call is asynchronous like the others; the work is ordered after
- * earlier work on `stream`, and later work on `stream` waits for all of it,
+ * The copies are pipelined with the compute: the chunks of q, k, v go to the device
+ * on h2d_stream as strided copies (causal: Q_0, K_0 V_0, Q_1, K_1 V_1, ...; else all
+ * of K, V first, then Q_0, Q_1, ...), every pair is launched as soon as both of its
+ * chunks are in, and a query chunk's merged result goes back on d2h_stream as soon
+ * as it is final. The call is asynchronous like the others; the work is ordered
+ * after earlier work on `stream`, and later work on `stream` waits for all of it,
  * including the last copy back.
  *
  *   q_h, k_h, v_h   HOST, bf16 [B][Hq][N][d], [B][Hkv][N][d]; page-locked memory

@@ -104,6 +104,23 @@ int64_t pair_heaviest_unit(const attn_pair_t& p, int causal) {
   return n < tiles ? n : tiles;
 }
 
+// Whether all of a pair's work units cost the same: even its first 256-row block sees
+// every key tile (the kernel's own test for its head-major unit order).
+bool pair_uniform(const attn_pair_t& p, int causal) {
+  const int64_t tiles = (p.kv_len + 127) / 128;
+  const int64_t lim0 = p.q_off + (p.q_len < 256 ? p.q_len : 256) - 1 - p.kv_off;
+  return !causal || lim0 >= (tiles - 1) * 128;
+}
+
+// Launch order of two pairs: heavier heaviest unit first; on a tie, pairs with equal
+// units before pairs with a causal cut, so that the grid's last units are the cut
+// pairs' light ones.
+bool goes_before(const attn_pair_t& a, const attn_pair_t& b, int causal) {
+  const int64_t ca = pair_heaviest_unit(a, causal), cb = pair_heaviest_unit(b, causal);
+  if (ca != cb) return ca > cb;
+  return pair_uniform(a, causal) && !pair_uniform(b, causal);
+}
+
 }  // namespace
 
 extern "C" {
@@ -238,9 +255,8 @@ attn_status_t attn_fwd_partial_batch(const void* q, const void* k, const void* v
   for (int i = 0; i < n_pairs; ++i) order[i] = i;
   for (int i = 1; i < n_pairs; ++i) {  // stable insertion sort, n_pairs <= 48
     const int x = order[i];
-    const int64_t cx = pair_heaviest_unit(pairs[x], causal);
     int j = i - 1;
-    while (j >= 0 && pair_heaviest_unit(pairs[order[j]], causal) < cx) {
+    while (j >= 0 && goes_before(pairs[x], pairs[order[j]], causal)) {
       order[j + 1] = order[j];
       --j;
     }
@@ -313,8 +329,19 @@ attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaStream_t sh = h2d_stream ? static_cast<cudaStream_t>(h2d_stream) : s;
   cudaStream_t sd = d2h_stream ? static_cast<cudaStream_t>(d2h_stream) : s;
-  // events: [0] start, [1] end, [2 + c] chunk c on the device, [2 + P + i] result i final
-  std::vector<cudaEvent_t> ev(2 + 2 * (size_t)n_chunks, nullptr);
+  const int P = n_chunks;
+
+  // Arrival points of the copies in: each point is a group of chunks whose arrival is
+  // marked by one event. Causal: Q_0, KV_0, Q_1, KV_1, ... - pair (i, kv < i) is ready
+  // once Q_i is in, the diagonal pair (i, i) once KV_i is, so when the last chunk
+  // arrives only one diagonal pair is left to compute. Non-causal (every query chunk
+  // needs every key/value chunk): KV_0 .. KV_{P-1}, then Q_0, Q_1, ... - query chunk
+  // i is ready once Q_i is in, and results leave while later Q chunks still arrive.
+  const int n_points = 2 * P;
+  auto q_point = [&](int i) { return causal ? 2 * i : P + i; };
+  auto kv_point = [&](int c) { return causal ? 2 * c + 1 : c; };
+  // events: [0] start, [1] end, [2 + t] arrival point t, [2 + n_points + i] result i final
+  std::vector<cudaEvent_t> ev(2 + (size_t)n_points + P, nullptr);
   auto release = [&]() {
     for (cudaEvent_t e : ev)
       if (e) cudaEventDestroy(e);  // resources are released once pending work completes
@@ -339,55 +366,83 @@ attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v
   // (the copies back wait for events recorded on `stream`, so they follow it anyway)
   after(sh, ev[0], s);
 
-  // host -> device: chunk c of k, v, q as strided copies (B*H runs of C rows)
+  // host -> device, one arrival point at a time: strided copies (B*H runs of C rows)
   const size_t pitch = (size_t)N * d * 2, width = (size_t)C * d * 2;
-  for (int c = 0; c < n_chunks && st == ATTN_OK; ++c) {
+  auto copy_in = [&](void* dst, const void* src, int c, uint64_t runs) {
     const size_t off = (size_t)c * width;
-    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(k_d) + off, pitch,
-                              static_cast<const char*>(k_h) + off, pitch, width, bhkv,
+    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(dst) + off, pitch,
+                              static_cast<const char*>(src) + off, pitch, width, runs,
                               cudaMemcpyHostToDevice, sh));
-    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(v_d) + off, pitch,
-                              static_cast<const char*>(v_h) + off, pitch, width, bhkv,
-                              cudaMemcpyHostToDevice, sh));
-    cuda_ok(cudaMemcpy2DAsync(static_cast<char*>(q_d) + off, pitch,
-                              static_cast<const char*>(q_h) + off, pitch, width, bh,
-                              cudaMemcpyHostToDevice, sh));
-    if (st == ATTN_OK && sh != s) cuda_ok(cudaEventRecord(ev[2 + c], sh));
+  };
+  for (int t = 0; t < n_points && st == ATTN_OK; ++t) {
+    for (int c = 0; c < P; ++c) {
+      if (kv_point(c) == t) {
+        copy_in(k_d, k_h, c, bhkv);
+        copy_in(v_d, v_h, c, bhkv);
+      }
+      if (q_point(c) == t) copy_in(q_d, q_h, c, bh);
+    }
+    if (st == ATTN_OK && sh != s) cuda_ok(cudaEventRecord(ev[2 + t], sh));
   }
 
-  // per query chunk: its partials in one launch, their merge, and the copy back
+  // Pairs launch at their arrival point (one batched launch per point); a query
+  // chunk's partials go to partial slot j for its j-th key/value chunk in ring order
+  // (chunk (i - j) mod P), are merged in that order once its last pair has run, and the
+  // result goes back. A query chunk's pairs all run between two of its own points, and
+  // chunks finish in order, so P partial slots serve every chunk.
+  auto visits = [&](int i, int* kv_of_slot) {
+    int nv = 0;
+    for (int step = 0; step < P; ++step) {
+      const int kv = ((i - step) % P + P) % P;
+      if (causal && kv > i) continue;
+      kv_of_slot[nv++] = kv;
+    }
+    return nv;
+  };
   attn_pair_t pairs[ATTN_MAX_BATCH_PAIRS];
   const float* po[ATTN_MAX_BATCH_PAIRS];
   const float* pl[ATTN_MAX_BATCH_PAIRS];
-  for (int qi = 0; qi < n_chunks && st == ATTN_OK; ++qi) {
-    if (sh != s && !cuda_ok(cudaStreamWaitEvent(s, ev[2 + (causal ? qi : n_chunks - 1)], 0)))
-      break;
-    float* o_i = o_d + (size_t)qi * slot_rows * d;
-    float* l_i = lse_d + (size_t)qi * slot_rows;
-    int nv = 0;
-    for (int step = 0; step < n_chunks; ++step) {
-      const int kv = ((qi - step) % n_chunks + n_chunks) % n_chunks;
-      if (causal && kv > qi) continue;
-      pairs[nv] = attn_pair_t{qi * C, C, kv * C, C, qi * C, kv * C, nullptr, nullptr};
-      ++nv;
+  int kv_of_slot[ATTN_MAX_BATCH_PAIRS];
+  for (int t = 0; t < n_points && st == ATTN_OK; ++t) {
+    int np = 0;
+    int finished = -1;  // the query chunk whose last pair runs at this point, if any
+    for (int i = 0; i < P; ++i) {
+      const int nv = visits(i, kv_of_slot);
+      int last = -1;
+      for (int j = 0; j < nv; ++j) {
+        const int kv = kv_of_slot[j];
+        const int ready = q_point(i) > kv_point(kv) ? q_point(i) : kv_point(kv);
+        last = ready > last ? ready : last;
+        if (ready != t) continue;
+        float* o_j = nv == 1 ? o_d + (size_t)i * slot_rows * d : ws_o + (size_t)j * slot_rows * d;
+        float* l_j = nv == 1 ? lse_d + (size_t)i * slot_rows : ws_lse + (size_t)j * slot_rows;
+        pairs[np++] = attn_pair_t{i * C, C, kv * C, C, i * C, kv * C, o_j, l_j};
+      }
+      if (last == t) finished = i;
     }
-    for (int j = 0; j < nv; ++j) {
-      pairs[j].o = nv == 1 ? o_i : ws_o + (size_t)j * slot_rows * d;
-      pairs[j].lse = nv == 1 ? l_i : ws_lse + (size_t)j * slot_rows;
-      po[j] = pairs[j].o;
-      pl[j] = pairs[j].lse;
-    }
-    st = attn_fwd_partial_batch(q_d, k_d, v_d, B, Hq, Hkv, N, N, d, causal, scale, pairs, nv, 0,
+    if (np == 0) continue;
+    if (sh != s && !cuda_ok(cudaStreamWaitEvent(s, ev[2 + t], 0))) break;
+    st = attn_fwd_partial_batch(q_d, k_d, v_d, B, Hq, Hkv, N, N, d, causal, scale, pairs, np, 0,
                                 stream);
-    if (st == ATTN_OK && nv > 1)
+    if (st != ATTN_OK || finished < 0) continue;
+    const int i = finished;
+    float* o_i = o_d + (size_t)i * slot_rows * d;
+    float* l_i = lse_d + (size_t)i * slot_rows;
+    const int nv = visits(i, kv_of_slot);
+    if (nv > 1) {
+      for (int j = 0; j < nv; ++j) {
+        po[j] = ws_o + (size_t)j * slot_rows * d;
+        pl[j] = ws_lse + (size_t)j * slot_rows;
+      }
       st = attn_merge(po, pl, nv, o_i, l_i, (int64_t)slot_rows, d, stream);
-    if (st != ATTN_OK) break;
-    if (sd != s && !(cuda_ok(cudaEventRecord(ev[2 + n_chunks + qi], s)) &&
-                     cuda_ok(cudaStreamWaitEvent(sd, ev[2 + n_chunks + qi], 0))))
+      if (st != ATTN_OK) break;
+    }
+    if (sd != s && !(cuda_ok(cudaEventRecord(ev[2 + n_points + i], s)) &&
+                     cuda_ok(cudaStreamWaitEvent(sd, ev[2 + n_points + i], 0))))
       break;
-    cuda_ok(cudaMemcpyAsync(o_h + (size_t)qi * slot_rows * d, o_i, slot_rows * d * 4,
+    cuda_ok(cudaMemcpyAsync(o_h + (size_t)i * slot_rows * d, o_i, slot_rows * d * 4,
                             cudaMemcpyDeviceToHost, sd));
-    cuda_ok(cudaMemcpyAsync(lse_h + (size_t)qi * slot_rows, l_i, slot_rows * 4,
+    cuda_ok(cudaMemcpyAsync(lse_h + (size_t)i * slot_rows, l_i, slot_rows * 4,
                             cudaMemcpyDeviceToHost, sd));
   }
   // later work on `stream` waits for the last copy back
