@@ -32,3 +32,28 @@ def test_one_rank_ring_equals_single_pass(causal):
         assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
     finally:
         dist.destroy_process_group()
+
+
+def test_one_rank_ulysses_and_grid_equal_single_pass():
+    """Ulysses' all-to-all exchanges and the 1 x 1 ATTENTION2D grid on one NCCL rank:
+    the library's kernels behind them give attn_fwd's result bit for bit."""
+    import torch.distributed as dist
+
+    import online_softmax_exact_b200 as osx
+    from online_softmax_exact_b200.grid2d_dist import grid2d_attention_dist
+    from online_softmax_exact_b200.ulysses_dist import ulysses_attention_dist
+
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1)
+    try:
+        q = randn_bf16((2, 4, 700, 64), 27, 0).cuda()
+        k = randn_bf16((2, 2, 700, 64), 27, 1).cuda()
+        v = randn_bf16((2, 2, 700, 64), 27, 2).cuda()
+        o_ref, l_ref = osx.attn_fwd(q, k, v, causal=True)
+        o_u, l_u = ulysses_attention_dist(q, k, v, causal=True)
+        o_g, l_g = grid2d_attention_dist(q, k, v, p_q=1, p_kv=1, causal=True)
+        torch.cuda.synchronize()
+        assert osx.attn_device_status() == osx.ATTN_OK
+        assert torch.equal(o_u, o_ref) and torch.equal(l_u, l_ref)
+        assert torch.equal(o_g, o_ref) and torch.equal(l_g, l_ref)
+    finally:
+        dist.destroy_process_group()
