@@ -114,11 +114,19 @@ bool pair_uniform(const attn_pair_t& p, int causal) {
 
 // Launch order of two pairs: heavier heaviest unit first; on a tie, pairs with equal
 // units before pairs with a causal cut, so that the grid's last units are the cut
-// pairs' light ones.
+// pairs' light ones; among pairs with equal units, those that read the same key/value
+// chunk side by side (the kernel then runs them head by head across the group).
 bool goes_before(const attn_pair_t& a, const attn_pair_t& b, int causal) {
   const int64_t ca = pair_heaviest_unit(a, causal), cb = pair_heaviest_unit(b, causal);
   if (ca != cb) return ca > cb;
-  return pair_uniform(a, causal) && !pair_uniform(b, causal);
+  const bool ua = pair_uniform(a, causal), ub = pair_uniform(b, causal);
+  if (ua != ub) return ua;
+  if (ua) {
+    if (a.kv_start != b.kv_start) return a.kv_start < b.kv_start;
+    if (a.kv_len != b.kv_len) return a.kv_len < b.kv_len;
+    if (a.q_len != b.q_len) return a.q_len < b.q_len;
+  }
+  return false;
 }
 
 }  // namespace

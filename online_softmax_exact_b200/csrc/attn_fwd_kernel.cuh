@@ -53,6 +53,9 @@ struct PairDesc {
   int q_row0, kv_row0;       // tensor-map row of the chunks' first rows
   int Nq, Nkv;               // chunk lengths
   int uniform;               // every unit visits all key tiles (no causal truncation)
+  // Uniform pairs that read the same key/value chunk with the same shapes form a group
+  // (consecutive in the table): pairs group_first .. group_first + group_n - 1.
+  int group_first, group_n;
 };
 
 struct FwdParams {
@@ -104,11 +107,12 @@ __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
 }
 
 // A work unit: 256 query rows (two 128-row tiles) of one (batch, head) of one pair.
-// Units are numbered pair by pair (pairs in launch order, heaviest first). Within a pair
-// whose units all cost the same, heads are outermost, so that the CTAs running at one
-// time share the key/value tiles of a few heads in L2; otherwise row blocks go from the
-// last to the first (heaviest first under the causal mask) with heads innermost, query
-// heads sharing a key/value head side by side.
+// Units are numbered pair by pair (pairs in launch order, heaviest first). Within a
+// group of pairs whose units all cost the same and that read one key/value chunk,
+// heads are outermost (then pair, then row block), so that the CTAs running at one
+// time share the key/value tiles of a few heads in L2; in other pairs row blocks go
+// from the last to the first (heaviest first under the causal mask) with heads
+// innermost, query heads sharing a key/value head side by side.
 struct Unit {
   int pair, qp, bh;
   int n;  // key tiles the unit visits
@@ -118,18 +122,26 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit un;
   int i = 0;
   while (i + 1 < p.n_pairs && u >= p.unit_end[i]) ++i;
-  const int ul = u - (i ? p.unit_end[i - 1] : 0);
-  const PairDesc& pr = p.pair[i];
-  const int n_qpairs = (pr.Nq + 255) / 256;
-  const int n_kv_tiles = (pr.Nkv + 127) / 128;
-  un.pair = i;
-  if (pr.uniform) {
-    un.bh = ul / n_qpairs;
-    un.qp = n_qpairs - 1 - ul % n_qpairs;
+  const PairDesc& pi = p.pair[i];
+  const int n_qpairs = (pi.Nq + 255) / 256;  // the same for every pair of a group
+  if (pi.uniform) {
+    // heads outermost across the whole group, so that the CTAs running at one time
+    // share the key/value tiles of a few heads in L2 for every query chunk at once
+    const int first = pi.group_first;
+    const int ug = u - (first ? p.unit_end[first - 1] : 0);
+    const int per_head = pi.group_n * n_qpairs;
+    un.bh = ug / per_head;
+    const int rem = ug - un.bh * per_head;
+    un.pair = first + rem / n_qpairs;
+    un.qp = n_qpairs - 1 - rem % n_qpairs;
   } else {
+    const int ul = u - (i ? p.unit_end[i - 1] : 0);
+    un.pair = i;
     un.qp = n_qpairs - 1 - ul / p.BH;
     un.bh = ul % p.BH;
   }
+  const PairDesc& pr = p.pair[un.pair];
+  const int n_kv_tiles = (pr.Nkv + 127) / 128;
   // all key tiles, or under the causal mask those up to the last key visible to the
   // unit's last valid row; 0 means no row of the unit sees any key
   un.n = n_kv_tiles;

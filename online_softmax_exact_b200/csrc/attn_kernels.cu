@@ -123,6 +123,16 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
       const long long lim0 = s.q_off + last_row0 - s.kv_off;
       d.uniform = (!a.causal || lim0 >= (tiles - 1) * 128) ? 1 : 0;
     }
+    // a uniform pair joins the previous pair's group if that one is uniform too and
+    // reads the same key/value rows with the same shapes
+    d.group_first = i;
+    d.group_n = 1;
+    if (i > 0 && d.uniform && p.pair[i - 1].uniform && p.pair[i - 1].kv_row0 == d.kv_row0 &&
+        p.pair[i - 1].Nkv == d.Nkv && p.pair[i - 1].Nq == d.Nq) {
+      d.group_first = p.pair[i - 1].group_first;
+      d.group_n = i - d.group_first + 1;
+      for (int g = d.group_first; g < i; ++g) p.pair[g].group_n = d.group_n;
+    }
     if ((reinterpret_cast<uintptr_t>(s.o) % 32) != 0) p.o_vec8 = 0;
     units += ((s.q_len + 255) / 256) * (long long)p.BH;
     if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
