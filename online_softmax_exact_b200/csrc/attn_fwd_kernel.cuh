@@ -497,7 +497,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (__all_sync(0xffffffffu, !need_mask && m != -INFINITY)) {
           // Common case: exponentiate against the current running maximum while the tile
           // maximum is reduced alongside; the maximum only moves when a row's tile maximum
-          // exceeds it by more than 8 (log2 units), and then the warp redoes P.
+          // exceeds it by more than 8 (log2 units). It then moves up by a whole number k
+          // of octaves (k >= the excess), so the P already stored only needs scaling by
+          // 2^-k, which is exact; P is recomputed only if it may have overflowed.
           float mx;
           sum = softmax_half<false, true>(s, tS, c, m, climit, &mx);
           xch_mine[par * 256] = mx;
@@ -505,11 +507,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mx = fmaxf(mx, xch_other[par * 256]);
           const float m_tile = mx * c;
           const bool grow = m_tile > m + 8.0f;
-          m_new = grow ? m_tile : m;
-          alpha = grow ? ex2_approx(m - m_new) : 1.f;
+          m_new = m;
+          alpha = 1.f;
           if (__any_sync(0xffffffffu, grow)) {
-            tmem_st_wait();  // the first P stores land before they are overwritten
-            sum = softmax_half<false, false>(s, tS, c, m_new, climit, nullptr);
+            const float excess = m_tile - m;
+            const bool big = grow && excess > 100.0f;  // P against m may have overflowed
+            const int k = (grow && !big) ? (int)ceilf(excess) : 0;
+            m_new = grow ? (big ? m_tile : m + (float)k) : m;
+            alpha = big ? ex2_approx(m - m_new) : exp2_neg_int(k);
+            tmem_st_wait();  // the first P stores land before they are read back
+            if (__any_sync(0xffffffffu, big)) {
+              sum = softmax_half<false, false>(s, tS, c, m_new, climit, nullptr);
+            } else {
+              const uint32_t a2 = pack_bf16x2(alpha, alpha);
+#pragma unroll 1
+              for (int q2 = 0; q2 < 2; ++q2) {  // rare: kept small rather than fast
+                uint32_t pv[16];
+                tmem_ld16(tS + q2 * 16, pv);
+                tmem_ld_wait(pv);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pv[i] = mul_bf16x2(pv[i], a2);
+                tmem_st16(tS + q2 * 16, pv);
+              }
+              sum *= alpha;
+            }
           }
         } else {
           float mx = -INFINITY;

@@ -298,6 +298,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return d;
 }
 
+// a * b for packed bf16 pairs (round to nearest; exact when b is a power of two and
+// the result stays normal)
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 2^-k as a float, exactly, for an integer 0 <= k <= 126
+__device__ __forceinline__ float exp2_neg_int(int k) { return __int_as_float((127 - k) << 23); }
+
 // 256-bit global store of 8 floats (address 32-byte aligned)
 __device__ __forceinline__ void st_global_v8(float* p, float a0, float a1, float a2, float a3,
                                              float a4, float a5, float a6, float a7) {
