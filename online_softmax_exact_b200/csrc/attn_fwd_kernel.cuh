@@ -8,9 +8,10 @@
 // end. Scores never leave the SM.
 //
 // B200 mapping (our design, not the page's):
-//   * one CTA per SM (persistent), work unit = 256 query rows of one (batch, head),
-//     held as two 128-row tiles in ping-pong: the tensor core works on one tile while
-//     the other tile's softmax runs;
+//   * one CTA per SM (persistent), work unit = 256 query rows of one (batch, head) of
+//     one (query chunk, key/value chunk) pair, held as two 128-row tiles in ping-pong:
+//     the tensor core works on one tile while the other tile's softmax runs; a launch
+//     carries up to kMaxPairs pairs, their units in one static schedule;
 //   * warp 16 issues TMA loads (Q tiles once per unit, K and V tiles through a ring of
 //     shared-memory stages, 128-byte swizzle);
 //   * warp 17 owns tensor memory and issues tcgen05.mma from one thread:
@@ -25,8 +26,10 @@
 //     is the running maximum m, moved only when a tile maximum exceeds it by more than
 //     8 (log2 units); exactness is kept because numerator and denominator share the
 //     same base. In the common case the exponentials are computed against the current
-//     m while the tile maximum is reduced alongside, and redone only if m moves; when
-//     m moves the threads rescale their halves of O in TMEM;
+//     m while the tile maximum is reduced alongside; if m moves, it moves by a whole
+//     number of octaves, so the P already written is rescaled by an exact power of two
+//     (recomputed only after a jump so large that it may have overflowed), and the
+//     threads rescale their halves of O in TMEM;
 //   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32; in accumulate mode
 //     the result is first combined with the normalised partial (O_acc, LSE_acc) already
 //     in o/lse by the log-sum-exp rule of the merge (weights e^(LSE - max LSE)).
