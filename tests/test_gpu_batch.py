@@ -91,3 +91,33 @@ def test_batched_ring_32k(osx, fused):
     rt = torch.from_numpy(rows).cuda()
     o_ref, l_ref = oracle.attention_rows(q, k, v, causal=True, scale=w.scale, rows=rows)
     compare(to_np(o.index_select(2, rt)), to_np(lse.index_select(2, rt)), o_ref, l_ref)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_grouped_pairs_equal_single_pair_calls(osx, causal):
+    """Pairs with equal units that read one key/value chunk run as a group, head by head
+    across the group; each pair's result is still the single call's, bit for bit."""
+    d = 128
+    q = randn_bf16((2, 4, 2048, d), 71, 0)
+    k = randn_bf16((2, 2, 2048, d), 71, 1)
+    v = randn_bf16((2, 2, 2048, d), 71, 2)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    spec = [(1024, 256, 512, 384), (512, 256, 512, 384), (1280, 256, 512, 384),
+            (1536, 256, 512, 384), (0, 256, 512, 384), (1792, 256, 512, 384),
+            (1792, 256, 0, 384)]
+    pairs, singles = [], []
+    for qs, ql, ks, kl in spec:
+        o1, l1 = osx.attn_fwd_partial(qg, kg, vg, q_start=qs, q_len=ql, kv_start=ks,
+                                      kv_len=kl, causal=causal)
+        singles.append((o1, l1))
+        pairs.append(dict(q_start=qs, q_len=ql, kv_start=ks, kv_len=kl,
+                          o=torch.empty_like(o1), lse=torch.empty_like(l1)))
+    osx.attn_fwd_partial_batch(qg, kg, vg, pairs, causal=causal)
+    assert osx.attn_device_status() == osx.ATTN_OK
+    for pr, (o1, l1) in zip(pairs, singles):
+        assert torch.equal(pr["o"], o1) and torch.equal(pr["lse"], l1)
+    pr = pairs[3]
+    o_ref, l_ref = oracle.attention(q[:, :, 1536:1792].contiguous(),
+                                    k[:, :, 512:896].contiguous(), v[:, :, 512:896].contiguous(),
+                                    causal=causal, scale=d ** -0.5, q_off=1536, kv_off=512)
+    compare(to_np(pr["o"]), to_np(pr["lse"]), o_ref, l_ref)

@@ -103,6 +103,25 @@ def test_fwd_rescale_stress(osx, d):
         compare(o, lse, o_ref, l_ref)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_running_max_jumps(osx, d):
+    """Rows whose maximum jumps by tens of octaves (P rescaled in place by a power of
+    two) and by hundreds (P recomputed) on later key tiles, with and without the mask."""
+    N = 640
+    q, k, v = inputs(1, 2, 2, N, N, d, seed=123)
+    q = q.clone()
+    k = k.clone()
+    q[..., 0] = 8.0
+    # with q[0] = 8, k[0] = J ln2 sqrt(d) / 8 lifts that key's logit by about J octaves
+    # (the others stay within a few octaves of 0)
+    for j, octaves in ((200, 30.0), (250, 60.0), (400, 200.0), (600, 800.0)):
+        k[:, :, j, 0] = octaves * math.log(2.0) * math.sqrt(d) / 8.0
+    for causal in (False, True):
+        o_ref, l_ref = oracle.attention(q, k, v, causal=causal, scale=1 / math.sqrt(d))
+        o, lse = run_fwd(osx, q, k, v, causal, 1 / math.sqrt(d))
+        compare(o, lse, o_ref, l_ref)
+
+
 def test_fwd_zero_scale_is_mean_of_visible_values(osx):
     q, k, v = inputs(1, 2, 2, 300, 300, 128, seed=5)
     o, lse = run_fwd(osx, q, k, v, True, 0.0)
