@@ -33,10 +33,14 @@
  * inputs, a negative or non-finite scale, and offsets/leading dimensions that do
  * not fit give ATTN_ERR_INVALID_ARG. Shapes the kernels are not built for (d other
  * than 64 or 128, more than ATTN_MAX_MERGE_PARTS parts, sizes beyond the tensor-map
- * limits) give ATTN_ERR_UNSUPPORTED. A failed CUDA call gives ATTN_ERR_CUDA. A
- * device-side wait that ran out of time is reported by attn_device_status as
- * ATTN_ERR_TIMEOUT; it never traps. NaN or Inf inside q, k, v is not checked and
- * gives unspecified results.
+ * limits) give ATTN_ERR_UNSUPPORTED. A failed CUDA call gives ATTN_ERR_CUDA. NaN or
+ * Inf inside the rows a call attends is not checked and gives unspecified results.
+ *
+ * Device-side failures. Every wait inside the kernels is bounded (4 s of wall-clock
+ * time). A wait that runs out stops the kernel early, leaves its outputs unspecified
+ * and is recorded in a per-device status word; the launch itself has already returned
+ * ATTN_OK by then. Results therefore count only once attn_device_status has reported
+ * ATTN_OK for the stream they were computed on. Nothing traps or faults.
  */
 #ifndef ATTN_H
 #define ATTN_H
@@ -154,8 +158,11 @@ attn_status_t attn_fwd_partial_acc(const void* q, const void* k_chunk, const voi
  *   q      device, bf16 parent [B][Hq][q_ld][d];  k, v: parents [B][Hkv][kv_ld][d]
  *   pairs  HOST array of n_pairs (1 .. ATTN_MAX_BATCH_PAIRS) pair descriptions; every
  *          chunk must lie inside its parent; no two pairs' outputs may overlap
- *   other arguments as for attn_fwd_partial. Keys of a parent outside a pair's chunk
- *   are masked out (never weighted), and must be finite like all inputs.
+ *   other arguments as for attn_fwd_partial. Rows of a parent outside a pair's chunks
+ *   may hold anything, NaN and Inf included (uninitialised memory, or a copy still in
+ *   flight): a pair reads them into its last tiles but they never reach its result
+ *   (keys there are masked, their value rows are zeroed on chip before P.V, and query
+ *   rows there are not stored).
  */
 attn_status_t attn_fwd_partial_batch(const void* q, const void* k, const void* v, int B,
                                      int Hq, int Hkv, int64_t q_ld, int64_t kv_ld, int d,
@@ -207,7 +214,9 @@ attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_pa
  *                   lets the copies overlap (pageable memory works, unoverlapped)
  *   o_h, lse_h      HOST, fp32 chunk-major [n_chunks][B][Hq][C][d] and
  *                   [n_chunks][B][Hq][C] (written)
- *   q_d, k_d, v_d   DEVICE staging, same shapes as q_h, k_h, v_h (16-byte aligned)
+ *   q_d, k_d, v_d   DEVICE staging, same shapes as q_h, k_h, v_h (16-byte aligned);
+ *                   their contents on entry do not matter (a pair may run before the
+ *                   neighbouring chunk has arrived; see attn_fwd_partial_batch)
  *   o_d, lse_d      DEVICE, same shapes as o_h, lse_h (o_d 32-byte aligned)
  *   ws_o, ws_lse    DEVICE partial buffers, ws_slots slots of [B][Hq][C][d] and
  *                   [B][Hq][C] (ws_o 32-byte aligned); ws_slots must be at least
@@ -216,6 +225,9 @@ attn_status_t attn_merge(const float* const* o_parts, const float* const* lse_pa
  *   n_chunks        1 .. ATTN_MAX_BATCH_PAIRS, dividing N
  *   h2d_stream, d2h_stream  streams for the two copy directions (NULL: `stream`)
  *   other arguments as for attn_fwd. Device buffers must not overlap each other.
+ * The host buffers are read and written by copies that run after the call returns:
+ * they must stay allocated (and q_h, k_h, v_h unchanged) until `stream` has passed
+ * this call's work.
  */
 attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v_h,
                                  float* o_h, float* lse_h, void* q_d, void* k_d, void* v_d,
@@ -245,9 +257,10 @@ attn_status_t attn_debug_inject(int status, int count);
  * attn_debug_wait_timeout - failure-path check for tests: launches one tiny kernel
  * whose single waiting thread waits, through the same bounded mbarrier wait the
  * attention kernel uses, on a barrier that nothing arrives on, with a limit of
- * limit_cycles SM clock cycles (1 .. 2^31). The wait runs out, the kernel records
- * ATTN_ERR_TIMEOUT in the device status word (see attn_device_status) and returns;
- * the device stays usable. Nothing traps or faults.
+ * limit_cycles SM clock cycles at the device's peak clock (1 .. 2^31; converted to
+ * wall-clock time, as the kernels' own limit is). The wait runs out, the kernel
+ * records ATTN_ERR_TIMEOUT in the device status word (see attn_device_status) and
+ * returns; the device stays usable. Nothing traps or faults.
  */
 attn_status_t attn_debug_wait_timeout(int64_t limit_cycles, void* stream);
 

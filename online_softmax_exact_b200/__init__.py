@@ -259,6 +259,19 @@ class RingHostBuffers:
 
 _copy_streams: dict = {}
 
+# Host tensors of attn_ring_fwd_host calls whose copies may still be queued: each entry
+# holds an event recorded after the call's work and the tensors it reads or writes, so
+# that a temporary (e.g. ``q.pin_memory()`` passed inline) is not freed, and its pinned
+# block reused, before the copies have run. Entries go once their event has completed.
+_inflight_host: list = []
+
+
+def _keep_alive_until_done(stream, tensors) -> None:
+    _inflight_host[:] = [(ev, ts) for ev, ts in _inflight_host if not ev.query()]
+    ev = torch.cuda.Event()
+    ev.record(stream)
+    _inflight_host.append((ev, tuple(tensors)))
+
 
 def _host_copy_streams(device: torch.device):
     if device.index not in _copy_streams:
@@ -321,6 +334,8 @@ def attn_ring_fwd_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, 
         _stream_handle(dev, s_main), _stream_handle(dev, h2d_stream),
         _stream_handle(dev, d2h_stream))
     _check(st, "attn_ring_fwd_host")
+    # later work on s_main waits for the last copy back (see attn.h)
+    _keep_alive_until_done(s_main, (q_h, k_h, v_h, o_h, lse_h))
     return o_h, lse_h
 
 

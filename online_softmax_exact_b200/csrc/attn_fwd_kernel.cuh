@@ -38,8 +38,14 @@
 // O_1 [384,384+D). Half h of P_t (bf16 pairs) overwrites S_t columns [64h, 64h+32),
 // inside that half's own score columns.
 //
+// Keys of the parent that lie past a pair's chunk but inside the tensor maps (pairs of a
+// batched launch) are read into the pair's last key tile. Their scores are masked, so
+// their P is exactly 0; the matching V rows are zeroed in shared memory before the P.V
+// MMA reads them, so that a non-finite value there cannot turn 0 * V into NaN.
+//
 // All mbarrier waits are bounded (see mbar_wait); on time-out the kernel records it in
-// the device status word, lets in-flight work drain, frees TMEM and returns.
+// the device status word, waits (bounded) for the copies it issued to land and for its
+// MMAs to complete, frees TMEM and returns.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -47,6 +53,9 @@
 namespace osx {
 
 constexpr int kMaxPairs = 48;
+
+// Limit of the final wait for in-flight copies (see the producer's drain).
+constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms
 
 // One (query chunk, key/value chunk) pair of a launch.
 struct PairDesc {
@@ -69,6 +78,7 @@ struct FwdParams {
   float scale_log2;    // scale * log2(e), >= 0
   int o_vec8;          // every O is 32-byte aligned: store rows with 256-bit stores
   int accumulate;      // o/lse hold a partial over other keys: fold this chunk into it
+  int kv_rows;         // rows of the K/V tensor maps (reads at or past them give zeros)
   int n_pairs;
   int unit_end[kMaxPairs];  // units of pairs 0..i: sum of ceil(Nq / 256) * BH
   PairDesc pair[kMaxPairs];
@@ -160,6 +170,30 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     }
   }
   return un;
+}
+
+// Row of the unit's last key tile from which the tile holds keys past the pair's chunk
+// that the tensor maps still cover (so TMA loaded real data there rather than zeros);
+// 128 when there are none.
+__device__ __forceinline__ int tail_rows_to_zero(const FwdParams& p, const Unit& un) {
+  const PairDesc& pr = p.pair[un.pair];
+  const int end = un.n * 128;  // rows the unit's key tiles span, from the chunk start
+  if (end <= pr.Nkv || pr.kv_row0 + pr.Nkv >= p.kv_rows) return 128;
+  return pr.Nkv - (un.n - 1) * 128;
+}
+
+// Zero rows [r0, 128) of a K/V tile in shared memory (D/64 boxes of 128 rows x 128
+// bytes; the 128-byte swizzle permutes 16-byte pieces within a row, so a row stays in
+// its own 128 bytes), then make the writes visible to the tensor core's operand reads.
+template <int D>
+__device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0) {
+#pragma unroll 1
+  for (int h = 0; h < D / 64; ++h) {
+    const uint32_t end = tile + (h + 1) * 16384;
+#pragma unroll 4
+    for (uint32_t a = tile + h * 16384 + r0 * 128; a < end; a += 16) st_shared_zero16(a);
+  }
+  fence_proxy_async_smem();
 }
 
 // One thread's half row of P for one 128-key tile (64 scores in s): x = S * c - m
@@ -272,6 +306,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // ---------------------------------------------------------------- TMA producer
       if (lane == 0) {
         int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
+        int k_arms = 0, v_arms = 0;  // K / V stage loads issued (for the final drain)
         bool ok = true;
         for (int r = 0; ok; ++r) {
           const int u = unit_for_round(r, blockIdx.x, G);
@@ -309,13 +344,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sbase + C::kKOff + ks * C::kTileBytes + h * 16384, &tmK, bar(B_KF + ks),
                           h * 64, pr.kv_row0 + j * 128, kvh);
+            ++k_arms;
             if (++ks == C::kStages) { ks = 0; kph ^= 1; }
             if (!(ok = mbar_wait(bar(B_VE + vs), vph ^ 1, abort_flag, p.status))) break;
             mbar_arrive_expect_tx(bar(B_VF + vs), C::kTileBytes);
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sbase + C::kVOff + vs * C::kTileBytes + h * 16384, &tmV, bar(B_VF + vs),
                           h * 64, pr.kv_row0 + j * 128, kvh);
+            ++v_arms;
             if (++vs == C::kStages) { vs = 0; vph ^= 1; }
+          }
+        }
+        // Wait until every copy issued has landed (the last armed phase of each full
+        // barrier has completed), so that no copy writes shared memory after the CTA
+        // exits. In a normal run they all have; after an abort some may still be in
+        // flight. Bounded; if it runs out, wait a fixed time instead.
+        bool drained = true;
+        if (qcount > 0) drained &= mbar_wait_drain(bar(B_QF), (qcount - 1) & 1, kDrainLimitNs);
+        for (int st = 0; st < C::kStages; ++st) {
+          const int kn = k_arms / C::kStages + (st < k_arms % C::kStages ? 1 : 0);
+          const int vn = v_arms / C::kStages + (st < v_arms % C::kStages ? 1 : 0);
+          if (kn > 0) drained &= mbar_wait_drain(bar(B_KF + st), (kn - 1) & 1, kDrainLimitNs);
+          if (vn > 0) drained &= mbar_wait_drain(bar(B_VF + st), (vn - 1) & 1, kDrainLimitNs);
+        }
+        if (!drained) {
+          const unsigned long long t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000ull) {
           }
         }
       }
@@ -363,8 +417,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int r = 0; ok; ++r) {
           const int u = unit_for_round(r, blockIdx.x, G);
           if (u >= n_units) break;
-          const int n = decode_unit(p, u).n;
+          const Unit un = decode_unit(p, u);
+          const int n = un.n;
           if (n == 0) continue;
+          // V rows of the last key tile to zero before its P.V (the last of the unit)
+          // reads them (128: none)
+          const int vz_row = tail_rows_to_zero(p, un);
           if (!(ok = mbar_wait(bar(B_QF), qcount & 1, abort_flag, p.status))) break;
           ++qcount;
           tc_fence_after();
@@ -396,6 +454,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mma_commit(bar(B_QE));
           // last P.V of the unit
           if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
+          if (vz_row < 128) zero_tile_rows<D>(sbase + C::kVOff + vs * C::kTileBytes, vz_row);
           for (int t = 0; t < 2; ++t) {
             if (!(ok = mbar_wait(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
             tc_fence_after();
@@ -670,16 +729,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {
-    // let in-flight tensor-core work and copies land before TMEM is freed
+    // let in-flight tensor-core work complete before TMEM is freed (the producer has
+    // already waited for its copies)
     if (warp == C::kWarpMma && lane == 0) {
       mma_commit(bar(B_DRAIN));
-      volatile int dummy = 0;
-      mbar_wait(bar(B_DRAIN), 0, &dummy, p.status);
-    }
-    if (warp == C::kWarpProducer && lane == 0) {
-      const unsigned long long t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < 200000ull) {
-      }
+      mbar_wait_drain(bar(B_DRAIN), 0, kDrainLimitNs);
     }
     __syncthreads();
   }

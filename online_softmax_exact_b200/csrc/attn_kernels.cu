@@ -19,7 +19,7 @@ __device__ unsigned g_device_status;
 // Failure-path check: one thread waits on an mbarrier that nothing arrives on, through
 // the same bounded wait the attention kernel uses, with a short limit. The wait runs
 // out, records kDevTimeout in the status word and the kernel returns.
-__global__ void wait_probe_kernel(unsigned* status, long long limit_cycles) {
+__global__ void wait_probe_kernel(unsigned* status, unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar_storage;
   __shared__ int abort_storage;
   if (threadIdx.x == 0) {
@@ -29,7 +29,7 @@ __global__ void wait_probe_kernel(unsigned* status, long long limit_cycles) {
   }
   __syncthreads();
   if (threadIdx.x == 0)
-    mbar_wait_limit(smem_u32(&bar_storage), 0, &abort_storage, status, limit_cycles);
+    mbar_wait_limit(smem_u32(&bar_storage), 0, &abort_storage, status, limit_ns);
   __syncthreads();
 }
 
@@ -40,6 +40,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  int clock_khz = 0;           // peak SM clock
   unsigned* status = nullptr;  // device address of g_device_status
 };
 
@@ -56,9 +57,11 @@ int device_info(DeviceInfo** out) {
   if (!di.ready) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!di.ready) {
-      int sms = 0;
+      int sms = 0, khz = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return ATTN_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0)
+        khz = 2000000;
       void* st = nullptr;
       if (cudaGetSymbolAddress(&st, g_device_status) != cudaSuccess) return ATTN_ERR_CUDA;
       if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -68,6 +71,7 @@ int device_info(DeviceInfo** out) {
                                (int)FwdCfg<128>::kSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
       di.num_sms = sms;
+      di.clock_khz = khz;
       di.status = static_cast<unsigned*>(st);
       di.ready = true;
     }
@@ -97,6 +101,7 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
   p.causal = a.causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.accumulate = a.accumulate;
+  p.kv_rows = static_cast<int>(a.kv_rows);
   p.n_pairs = a.n_pairs;
   p.o_vec8 = 1;
   long long units = 0;
@@ -202,7 +207,10 @@ int launch_wait_probe(long long limit_cycles, cudaStream_t stream) {
   DeviceInfo* di = nullptr;
   int rc = device_info(&di);
   if (rc != ATTN_OK) return rc;
-  wait_probe_kernel<<<1, 32, 0, stream>>>(di->status, limit_cycles);
+  // the device's wait limit is in nanoseconds: convert at the peak SM clock
+  const unsigned long long ns =
+      static_cast<unsigned long long>(limit_cycles) * 1000000ull / (unsigned)di->clock_khz + 1;
+  wait_probe_kernel<<<1, 32, 0, stream>>>(di->status, ns);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return ATTN_OK;

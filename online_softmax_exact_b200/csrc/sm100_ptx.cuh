@@ -16,10 +16,12 @@ enum : unsigned {
   kDevTimeout = 1u,  // an mbarrier wait exceeded its time limit
 };
 
-// Wait limit for any mbarrier: far above any legitimate wait (one tile of work is
-// microseconds), far below anything that looks like a hang. Counted in SM clock cycles
-// (cheap to read): 2^31 cycles is about 1.1 s at 1.9 GHz.
-constexpr long long kWaitLimitCycles = 1ll << 31;
+// Wait limit for any mbarrier, in nanoseconds of the global timer: far above any
+// legitimate wait (one tile of work is microseconds; a context time-sliced with other
+// processes on the same GPU is off the SMs for milliseconds at a time), far below
+// anything that looks like a hang. Wall-clock based, so that it does not depend on the
+// SM clock.
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 // Longest time a waiting thread stays parked in one try_wait before it re-checks the
 // abort flag and the limit; it wakes as soon as the phase completes.
 constexpr uint32_t kSuspendHintNs = 200000u;
@@ -68,18 +70,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete. The thread is parked
 // in try_wait (woken when the phase completes); between parks it checks the CTA-wide
-// abort flag and the cycle limit. Returns false if the flag is raised or the limit
-// passes (which raises the flag and records kDevTimeout in *status). Callers stop
-// their role on false.
+// abort flag and the time limit (global timer, nanoseconds). Returns false if the flag
+// is raised or the limit passes (which raises the flag and records kDevTimeout in
+// *status). Callers stop their role on false.
 __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
                                                 volatile int* abort_flag, unsigned* status,
-                                                long long limit_cycles) {
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
+  const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > limit_cycles) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(status, kDevTimeout);
       return false;
@@ -89,7 +91,18 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned* status) {
-  return mbar_wait_limit(bar, parity, abort_flag, status, kWaitLimitCycles);
+  return mbar_wait_limit(bar, parity, abort_flag, status, kWaitLimitNs);
+}
+
+// Bounded wait that ignores the abort flag (used while tearing down after an abort, to
+// let copies already in flight land). Returns false if the limit passes.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
+                                                unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  return true;
 }
 
 // ------------------------------------------------------------------------------------
@@ -130,6 +143,17 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
+}
+
+// 16 zero bytes to shared memory (generic proxy)
+__device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+}
+
+// Make this thread's earlier generic-proxy shared-memory writes visible to the async
+// proxy (tcgen05.mma operand reads, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Named barrier over `count` threads (a multiple of 32; id 0 is __syncthreads).
