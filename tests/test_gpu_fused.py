@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import TOL_MERGE, compare, to_np
+from parity_util import MERGE_LSE_ULPS, TOL_MERGE, compare, to_np
 from workloads import grid_merge_orders, randn_bf16
 
 pytestmark = pytest.mark.gpu
@@ -56,9 +56,15 @@ def test_accumulate_matches_the_merge_of_the_same_partials(osx):
     osx.attn_fwd_partial_acc(qg, kg, vg, q_start=0, q_len=512, kv_start=200, kv_len=312,
                              causal=False, o=acc_o, lse=acc_l)
     o64, l64 = oracle.merge([to_np(a[0]), to_np(b[0])], [to_np(a[1]), to_np(b[1])])
-    # the fused epilogue and the merge kernel round the same partial differently only
-    # through P's bf16 rounding being identical: both start from the same scores
-    compare(to_np(acc_o), to_np(acc_l), o64, l64, tol_o=1e-4, tol_lse=1e-5, rel_lse=True)
+    # The accumulating call forms the same scores, the same bf16 P and the same TMEM
+    # accumulator and denominator l as the plain partial b, so the two paths differ only
+    # in their final fp32 operations: the fused epilogue computes
+    # a * O_acc + (w_new / (w_acc + w_new) / l) * O_tmem, the merge w-weights the stored
+    # O_tmem / l. That is a handful of roundings of 2^-24 relative each, plus the
+    # ex2/lg2 approximations (2^-22 relative) in the weights, on |O| of order 1: far
+    # below 1e-5, so the merge's own bound applies.
+    compare(to_np(acc_o), to_np(acc_l), o64, l64, tol_o=TOL_MERGE, tol_lse=TOL_MERGE,
+            lse_ulps=MERGE_LSE_ULPS)
 
 
 def test_empty_accumulator_gives_the_plain_partial(osx):
@@ -71,7 +77,7 @@ def test_empty_accumulator_gives_the_plain_partial(osx):
     osx.attn_fwd_partial_acc(qg, kg, vg, q_start=0, q_len=384, kv_start=0, kv_len=384,
                              causal=True, o=o, lse=lse)
     compare(to_np(o), to_np(lse), to_np(plain[0]), to_np(plain[1]), tol_o=1e-6,
-            tol_lse=1e-6, rel_lse=True)
+            tol_lse=1e-6, lse_ulps=MERGE_LSE_ULPS)
 
 
 def test_chunk_hidden_by_the_mask_leaves_the_accumulator_unchanged(osx):

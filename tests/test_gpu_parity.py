@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import TOL_MERGE, compare, to_np
+from parity_util import MERGE_LSE_ULPS, TOL_MERGE, compare, to_np
 from workloads import get, randn_bf16, attention_inputs
 
 pytestmark = pytest.mark.gpu
@@ -65,7 +65,7 @@ def test_tiny_config_fwd_partials_merge(osx):
     om, lm = osx.attn_merge([p[0] for p in parts], [p[1] for p in parts])
     # merge of identical fp32 partials vs the fp64 merge of the same partials
     o64, l64 = oracle.merge([to_np(p[0]) for p in parts], [to_np(p[1]) for p in parts])
-    compare(to_np(om), to_np(lm), o64, l64, tol_o=TOL_MERGE, tol_lse=TOL_MERGE, rel_lse=True)
+    compare(to_np(om), to_np(lm), o64, l64, tol_o=TOL_MERGE, tol_lse=TOL_MERGE, lse_ulps=MERGE_LSE_ULPS)
     # chunked + merged vs the oracle, and vs the GPU single pass
     compare(to_np(om), to_np(lm), o_ref, l_ref)
     compare(to_np(om), to_np(lm), o, lse)
@@ -181,7 +181,7 @@ def test_merge_random_parts(osx, n, d):
     om, lm = osx.attn_merge(og, lg)
     o64, l64 = oracle.merge([t.double().numpy() for t in o_parts],
                             [t.double().numpy() for t in l_parts])
-    compare(to_np(om), to_np(lm), o64, l64, tol_o=TOL_MERGE, tol_lse=TOL_MERGE, rel_lse=True)
+    compare(to_np(om), to_np(lm), o64, l64, tol_o=TOL_MERGE, tol_lse=TOL_MERGE, lse_ulps=MERGE_LSE_ULPS)
     assert (to_np(om)[:7] == 0).all() and np.isneginf(to_np(lm)[:7]).all()
 
 
@@ -195,12 +195,12 @@ def test_merge_order_and_grouping_on_gpu(osx):
     for perm in itertools.permutations(range(4)):
         om, lm = osx.attn_merge([parts[i][0] for i in perm], [parts[i][1] for i in perm])
         compare(to_np(om), to_np(lm), to_np(ref[0]), to_np(ref[1]), tol_o=TOL_MERGE,
-                tol_lse=TOL_MERGE, rel_lse=True)
+                tol_lse=TOL_MERGE, lse_ulps=MERGE_LSE_ULPS)
     ab = osx.attn_merge([parts[0][0], parts[1][0]], [parts[0][1], parts[1][1]])
     cd = osx.attn_merge([parts[2][0], parts[3][0]], [parts[2][1], parts[3][1]])
     grouped = osx.attn_merge([ab[0], cd[0]], [ab[1], cd[1]])
     compare(to_np(grouped[0]), to_np(grouped[1]), to_np(ref[0]), to_np(ref[1]),
-            tol_o=1e-5, tol_lse=1e-5, rel_lse=True)
+            tol_o=1e-5, tol_lse=1e-5, lse_ulps=MERGE_LSE_ULPS)
     o_ref, l_ref = oracle.attention(q, k, v, causal=True, scale=128 ** -0.5)
     compare(to_np(ref[0]), to_np(ref[1]), o_ref, l_ref)
     single = osx.attn_fwd(qg, kg, vg, causal=True, scale=128 ** -0.5)
