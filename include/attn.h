@@ -237,6 +237,42 @@ attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v
                                  void* h2d_stream, void* d2h_stream);
 
 /*
+ * attn_ring_fwd_host_noalloc - attn_ring_fwd_host for callers that cannot allocate
+ * device memory. The pages have no counterpart of this call: it exists for programs in
+ * which cudaMalloc is not an option, for example code in a process whose device memory
+ * belongs to another allocator (a framework's caching allocator, a fixed per-component
+ * budget), or code on a latency-critical path where an allocation would synchronise the
+ * device. It takes the same host inputs and outputs as attn_ring_fwd_host and runs the
+ * same kernels in the same order (results are identical), but its device staging
+ * buffers and partial slots live in one fixed array of the library's own device data:
+ * it calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * The array holds ATTN_NOALLOC_SCRATCH_BYTES bytes, and every GPU on which the library
+ * is loaded keeps it until the process exits. A call needs, each piece rounded up to
+ * 256 bytes, with C = N / n_chunks and S = n_chunks if n_chunks > 1, else 0:
+ *     B*Hq*N*d*2 + 2 * B*Hkv*N*d*2 + B*Hq*N*d*4 + B*Hq*N*4 + S*B*Hq*C*d*4 + S*B*Hq*C*4
+ * bytes; a call that needs more returns ATTN_ERR_UNSUPPORTED before touching the
+ * device. Invalid arguments give ATTN_ERR_INVALID_ARG as for attn_ring_fwd_host.
+ *
+ * The first call on a device, with that device current, looks up the array's device
+ * address (once per device); make that first call before any stream capture. Every
+ * call shares the array, which keeps what the last call left in it; no part of it
+ * needs to start at zero, since a call writes every byte it uses before reading it.
+ * Calls whose work overlaps on the GPU race on the array: issue them on one stream
+ * (later calls on a stream wait for all the work of earlier ones, copies back
+ * included) or otherwise order them.
+ *
+ *   q_h, k_h, v_h, o_h, lse_h, B, Hq, Hkv, N, d, n_chunks, causal, scale, stream,
+ *   h2d_stream, d2h_stream: as for attn_ring_fwd_host
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (64ull * 1024ull * 1024ull)
+attn_status_t attn_ring_fwd_host_noalloc(const void* q_h, const void* k_h, const void* v_h,
+                                         float* o_h, float* lse_h, int B, int Hq, int Hkv,
+                                         int64_t N, int d, int n_chunks, int causal,
+                                         float scale, void* stream, void* h2d_stream,
+                                         void* d2h_stream);
+
+/*
  * attn_device_status - synchronise `stream` and report whether any kernel of this
  * library on the current device recorded a device-side failure since the last
  * reset (ATTN_ERR_TIMEOUT: a bounded wait ran out; the kernel then stopped its

@@ -22,6 +22,7 @@ from ._abi import (
     ATTN_ERR_TIMEOUT,
     ATTN_ERR_UNSUPPORTED,
     ATTN_MAX_MERGE_PARTS,
+    ATTN_NOALLOC_SCRATCH_BYTES,
     ATTN_OK,
     AttnError,
     load,
@@ -44,6 +45,7 @@ __all__ = [
     "attn_merge", "ATTN_MAX_BATCH_PAIRS", "attn_device_status", "attn_debug_inject",
     "attn_launch_count", "attn_status_string", "attn_version", "lib",
     "attn_debug_wait_timeout", "attn_ring_fwd_host", "RingHostBuffers",
+    "attn_ring_fwd_host_noalloc", "ATTN_NOALLOC_SCRATCH_BYTES",
 ]
 
 
@@ -335,6 +337,45 @@ def attn_ring_fwd_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, 
         _stream_handle(dev, d2h_stream))
     _check(st, "attn_ring_fwd_host")
     # later work on s_main waits for the last copy back (see attn.h)
+    _keep_alive_until_done(s_main, (q_h, k_h, v_h, o_h, lse_h))
+    return o_h, lse_h
+
+
+def attn_ring_fwd_host_noalloc(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, *,
+                               n_chunks: int, causal: bool, o_h: torch.Tensor,
+                               lse_h: torch.Tensor, scale: float | None = None,
+                               device=None, stream=None, h2d_stream=None, d2h_stream=None):
+    """attn_ring_fwd_host without device allocations: for callers that cannot allocate
+    device memory (the device buffers live in the library's fixed array of
+    ATTN_NOALLOC_SCRATCH_BYTES per GPU; see attn_ring_fwd_host_noalloc in attn.h).
+    The host outputs o_h / lse_h must be given (chunk-major, as attn_ring_fwd_host
+    returns them). Calls whose work overlaps on the GPU race: keep them on one stream."""
+    for t, n in ((q_h, "q_h"), (k_h, "k_h"), (v_h, "v_h")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 \
+                or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CPU bf16 tensor")
+    B, Hq, N, d = q_h.shape
+    Hkv = k_h.shape[1]
+    if n_chunks < 1 or N % n_chunks:
+        raise ValueError("the sequence length must split into equal chunks")
+    C = N // n_chunks
+    for t, shape, n in ((o_h, (n_chunks, B, Hq, C, d), "o_h"),
+                        (lse_h, (n_chunks, B, Hq, C), "lse_h")):
+        if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() \
+                or tuple(t.shape) != shape:
+            raise ValueError(f"{n} must be a contiguous CPU fp32 tensor of shape {shape}")
+    if scale is None:
+        scale = d ** -0.5
+    dev = torch.device(device) if device is not None else \
+        torch.device("cuda", torch.cuda.current_device())
+    s_main = stream if stream is not None else torch.cuda.current_stream(dev)
+    st = lib().attn_ring_fwd_host_noalloc(
+        q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
+        B, Hq, Hkv, N, d, n_chunks, int(bool(causal)), float(scale),
+        _stream_handle(dev, s_main),
+        _stream_handle(dev, h2d_stream) if h2d_stream is not None else None,
+        _stream_handle(dev, d2h_stream) if d2h_stream is not None else None)
+    _check(st, "attn_ring_fwd_host_noalloc")
     _keep_alive_until_done(s_main, (q_h, k_h, v_h, o_h, lse_h))
     return o_h, lse_h
 

@@ -18,6 +18,7 @@ ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_INJECTED = 5
 ATTN_MAX_MERGE_PARTS = 64
 ATTN_MAX_BATCH_PAIRS = 48
+ATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class AttnPair(ctypes.Structure):
@@ -58,6 +59,9 @@ SIGNATURES = {
     "attn_ring_fwd_host": (_i32, [_c_void_p] * 12 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32,
                                                      _i32, _f32, _c_void_p, _c_void_p,
                                                      _c_void_p]),
+    "attn_ring_fwd_host_noalloc": (_i32, [_c_void_p] * 5 + [_i32, _i32, _i32, _i64, _i32, _i32,
+                                                            _i32, _f32, _c_void_p, _c_void_p,
+                                                            _c_void_p]),
     "attn_device_status": (_i32, [_c_void_p, _i32]),
     "attn_debug_inject": (_i32, [_i32, _i32]),
     "attn_debug_wait_timeout": (_i32, [_i64, _c_void_p]),

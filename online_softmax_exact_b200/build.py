@@ -20,7 +20,7 @@ LIB = PKG / "libattn.so"
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
               "--expt-relaxed-constexpr"]
-SOURCES = ["attn_kernels.cu", "attn_api.cpp"]
+SOURCES = ["attn_kernels.cu", "attn_api.cpp", "attn_noalloc.cu"]
 DEPS = ["sm100_ptx.cuh", "tma_host.h", "attn_fwd_kernel.cuh", "attn_merge_kernel.cuh",
         "attn_internal.h"]
 

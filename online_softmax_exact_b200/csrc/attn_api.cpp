@@ -145,7 +145,7 @@ const char* attn_status_string(int status) {
   }
 }
 
-int attn_version(void) { return (1 << 16) | 1; }
+int attn_version(void) { return (1 << 16) | 2; }
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, float* o, float* lse, int B,
                        int Hq, int Hkv, int64_t N, int d, int causal, float scale, void* stream) {
