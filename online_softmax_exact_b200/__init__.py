@@ -45,7 +45,7 @@ __all__ = [
     "attn_merge", "ATTN_MAX_BATCH_PAIRS", "attn_device_status", "attn_debug_inject",
     "attn_launch_count", "attn_status_string", "attn_version", "lib",
     "attn_debug_wait_timeout", "attn_ring_fwd_host", "RingHostBuffers",
-    "attn_ring_fwd_host_noalloc", "ATTN_NOALLOC_SCRATCH_BYTES",
+    "attn_ring_fwd_host_noalloc", "ATTN_NOALLOC_SCRATCH_BYTES", "attn_debug_exp2",
 ]
 
 
@@ -388,6 +388,16 @@ def attn_device_status(stream=None, reset: bool = False) -> int:
 
 def attn_debug_inject(status: int, count: int) -> None:
     _check(lib().attn_debug_inject(int(status), int(count)), "attn_debug_inject")
+
+
+def attn_debug_exp2(x: torch.Tensor, *, use_poly: bool, stream=None) -> torch.Tensor:
+    """2^x of a CUDA fp32 tensor through the softmax's FMA-pipe polynomial (use_poly)
+    or through the exp unit (ex2.approx); for tests of the polynomial."""
+    _need(x, torch.float32, "x")
+    y = torch.empty_like(x)
+    _check(lib().attn_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), int(bool(use_poly)),
+                                 _stream_handle(x.device, stream)), "attn_debug_exp2")
+    return y
 
 
 def attn_debug_wait_timeout(limit_cycles: int, stream=None) -> None:

@@ -65,6 +65,7 @@ SIGNATURES = {
     "attn_device_status": (_i32, [_c_void_p, _i32]),
     "attn_debug_inject": (_i32, [_i32, _i32]),
     "attn_debug_wait_timeout": (_i32, [_i64, _c_void_p]),
+    "attn_debug_exp2": (_i32, [_c_void_p, _c_void_p, _i64, _i32, _c_void_p]),
     "attn_launch_count": (ctypes.c_uint64, []),
 }
 

@@ -459,6 +459,14 @@ attn_status_t attn_ring_fwd_host(const void* q_h, const void* k_h, const void* v
   return st;
 }
 
+attn_status_t attn_debug_exp2(const float* x, float* y, int64_t n, int use_poly, void* stream) {
+  if (!x || !y || n < 1 || (use_poly != 0 && use_poly != 1)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(y, 4)) return ATTN_ERR_INVALID_ARG;
+  if (overlap(span(x, (uint64_t)n * 4), span(y, (uint64_t)n * 4))) return ATTN_ERR_INVALID_ARG;
+  return static_cast<attn_status_t>(
+      osx::launch_exp2_probe(x, y, n, use_poly, static_cast<cudaStream_t>(stream)));
+}
+
 uint64_t attn_launch_count(void) { return osx::launch_count(); }
 
 }  // extern "C"

@@ -84,6 +84,19 @@ struct FwdParams {
   PairDesc pair[kMaxPairs];
 };
 
+// Pairs (bit i: pair i of every 16) of a thread's scores whose 2^x comes from the FMA
+// pipe in unmasked tiles, per head dimension. Measured on B200 (attn_fwd, TFLOP/s): at
+// D = 64, 2 pairs of 16 (12.5%) gain ~2% on large-logit inputs and ~1% on N(0,1); 4
+// pairs or more lose (the softmax is latency- and issue-bound, not exp-unit-bound, and
+// each polynomial costs ~5 instructions per value against 1). At D = 128 any share
+// loses 1-5%.
+#ifndef OSX_EMU_MASK_64
+#define OSX_EMU_MASK_64 0x0202u
+#endif
+#ifndef OSX_EMU_MASK_128
+#define OSX_EMU_MASK_128 0x0000u
+#endif
+
 template <int D>
 struct FwdCfg {
   static constexpr int kBM = 128;                    // rows per Q tile
@@ -111,6 +124,8 @@ struct FwdCfg {
   // holds 64 (4 * 104 + 64 = 5 * 96, the launch's total).
   static constexpr int kRegsSoftmax = 104;
   static constexpr int kRegsOther = 64;
+  // pairs of each 32-score block whose 2^x comes from the FMA pipe (bit i: pair i)
+  static constexpr uint32_t kEmu = (D == 64) ? OSX_EMU_MASK_64 : OSX_EMU_MASK_128;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 };
 
@@ -200,7 +215,10 @@ __device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0) {
 // (packed pairs), P = 2^x, written to TMEM as 32 columns of bf16 pairs at tP; returns
 // sum(P). Masked elements get x = -inf, for which ex2 gives exactly 0.
 // With kWithMax it also reduces the half-row maximum of the raw scores alongside.
-template <bool kMasked, bool kWithMax>
+// In unmasked tiles the pairs i (of 16 per 32 scores) with bit i of kEmu set take 2^x
+// from the FMA pipe (exp2_poly_f32x2) instead of the exp unit, so that the two pipes
+// share the exponentials.
+template <bool kMasked, bool kWithMax, uint32_t kEmu>
 __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP, float c,
                                               float m_use, int climit, float* tile_max) {
   float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -221,17 +239,24 @@ __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP,
       }
       float x0, x1, e0, e1;
       const uint64_t X = f2_fma(f2_pack(s0, s1), C2, NM2);
-      f2_unpack(X, x0, x1);
-      if (kMasked) {
-        if (q2 * 32 + 2 * i > climit) x0 = -INFINITY;
-        if (q2 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
+      uint64_t E;
+      if (!kMasked && ((kEmu >> i) & 1u)) {
+        E = exp2_poly_f32x2(X);
+        f2_unpack(E, e0, e1);
+      } else {
+        f2_unpack(X, x0, x1);
+        if (kMasked) {
+          if (q2 * 32 + 2 * i > climit) x0 = -INFINITY;
+          if (q2 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
+        }
+        e0 = ex2_approx(x0);
+        e1 = ex2_approx(x1);
+        E = f2_pack(e0, e1);
       }
-      e0 = ex2_approx(x0);
-      e1 = ex2_approx(x1);
       if (i & 1)
-        A23 = f2_add(A23, f2_pack(e0, e1));
+        A23 = f2_add(A23, E);
       else
-        A01 = f2_add(A01, f2_pack(e0, e1));
+        A01 = f2_add(A01, E);
       pk[i] = pack_bf16x2(e0, e1);
     }
     tmem_st16(tP + q2 * 16, pk);
@@ -563,7 +588,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // of octaves (k >= the excess), so the P already stored only needs scaling by
           // 2^-k, which is exact; P is recomputed only if it may have overflowed.
           float mx;
-          sum = softmax_half<false, true>(s, tS, c, m, climit, &mx);
+          sum = softmax_half<false, true, C::kEmu>(s, tS, c, m, climit, &mx);
           xch_mine[par * 256] = mx;
           if (!(ok = pair_sync())) break;
           mx = fmaxf(mx, xch_other[par * 256]);
@@ -579,7 +604,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             alpha = big ? ex2_approx(m - m_new) : exp2_neg_int(k);
             tmem_st_wait();  // the first P stores land before they are read back
             if (__any_sync(0xffffffffu, big)) {
-              sum = softmax_half<false, false>(s, tS, c, m_new, climit, nullptr);
+              sum = softmax_half<false, false, C::kEmu>(s, tS, c, m_new, climit, nullptr);
             } else {
               const uint32_t a2 = pack_bf16x2(alpha, alpha);
 #pragma unroll 1
@@ -618,8 +643,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // 1 when unchanged (also when both are -inf), 0 when m was -inf
           alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
           const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          sum = need_mask ? softmax_half<true, false>(s, tS, c, m_use, climit, nullptr)
-                          : softmax_half<false, false>(s, tS, c, m_use, climit, nullptr);
+          sum = need_mask ? softmax_half<true, false, 0u>(s, tS, c, m_use, climit, nullptr)
+                          : softmax_half<false, false, C::kEmu>(s, tS, c, m_use, climit, nullptr);
         }
         l = l * alpha + sum;
 

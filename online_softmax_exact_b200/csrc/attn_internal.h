@@ -37,6 +37,8 @@ int launch_merge(const float* const* o_parts, const float* const* lse_parts, int
                  float* o, float* lse, long long rows, int d, cudaStream_t stream);
 // Launches the failure-path check kernel (a bounded wait that must run out).
 int launch_wait_probe(long long limit_cycles, cudaStream_t stream);
+// Launches the exponential check kernel (y = 2^x by the polynomial or by ex2.approx).
+int launch_exp2_probe(const float* x, float* y, long long n, int use_poly, cudaStream_t stream);
 // Reads (and optionally clears) the device status word of the current device.
 int read_device_status(unsigned* out, int reset);
 uint64_t launch_count();

@@ -33,6 +33,26 @@ __global__ void wait_probe_kernel(unsigned* status, unsigned long long limit_ns)
   __syncthreads();
 }
 
+// Check of the exponentials the softmax uses: y = 2^x through the FMA-pipe polynomial
+// (use_poly != 0, two values per call as in the kernel) or through ex2.approx.
+__global__ void exp2_probe_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                  long long n, int use_poly) {
+  const long long stride = 2ll * gridDim.x * blockDim.x;
+  for (long long i = 2ll * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < n; i += stride) {
+    const bool two = i + 1 < n;
+    const float x0 = x[i], x1 = two ? x[i + 1] : 0.f;
+    float y0, y1;
+    if (use_poly) {
+      f2_unpack(exp2_poly_f32x2(f2_pack(x0, x1)), y0, y1);
+    } else {
+      y0 = ex2_approx(x0);
+      y1 = ex2_approx(x1);
+    }
+    y[i] = y0;
+    if (two) y[i + 1] = y1;
+  }
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -211,6 +231,18 @@ int launch_wait_probe(long long limit_cycles, cudaStream_t stream) {
   const unsigned long long ns =
       static_cast<unsigned long long>(limit_cycles) * 1000000ull / (unsigned)di->clock_khz + 1;
   wait_probe_kernel<<<1, 32, 0, stream>>>(di->status, ns);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return ATTN_OK;
+}
+
+int launch_exp2_probe(const float* x, float* y, long long n, int use_poly, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != ATTN_OK) return rc;
+  long long blocks = (n + 511) / 512;
+  if (blocks > (long long)di->num_sms * 8) blocks = (long long)di->num_sms * 8;
+  exp2_probe_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, y, n, use_poly);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return ATTN_OK;

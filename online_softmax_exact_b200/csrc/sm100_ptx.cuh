@@ -371,5 +371,46 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ------------------------------------------------------------------------------------
+// 2^x on the FMA pipe, two values at a time (no exp unit). Method: Cody and Waite's
+// argument reduction x = n + f with n = round(x), f in [-1/2, 1/2] (n taken with the
+// 1.5 * 2^23 shifter: adding it rounds x to an integer held in the low mantissa bits),
+// then 2^f from a degree-3 polynomial fitted here by the Remez exchange algorithm for
+// minimax relative error on [-1/2, 1/2] (csrc/exp2_poly_fit.py; max relative error
+// 7.5e-5), and 2^n applied by adding n to the result's exponent field. Inputs are
+// clamped below at -126 (2^-126 or a denormal comes out instead of a smaller value or
+// zero, so this is for unmasked scores only); inputs above 127 give garbage (callers
+// keep x <= 100). Horner's steps and the reduction run as packed f32x2 operations.
+// ------------------------------------------------------------------------------------
+constexpr float kExp2Shift = 12582912.0f;  // 1.5 * 2^23
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ uint64_t exp2_poly_f32x2(uint64_t X) {
+  float x0, x1;
+  f2_unpack(X, x0, x1);
+  const uint64_t Xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t SH = f2_pack(kExp2Shift, kExp2Shift);
+  const uint64_t T = f2_add(Xc, SH);  // low mantissa bits: n = round(x)
+  const uint64_t F = f2_sub(Xc, f2_sub(T, SH));
+  uint64_t P = f2_fma(F, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  P = f2_fma(P, F, f2_pack(kExp2C1, kExp2C1));
+  P = f2_fma(P, F, f2_pack(kExp2C0, kExp2C0));
+  float t0, t1, p0, p1;
+  f2_unpack(T, t0, t1);
+  f2_unpack(P, p0, p1);
+  // (bits(t) << 23) is n << 23: the shifter's own bits shift out of the word
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
 
 }  // namespace osx

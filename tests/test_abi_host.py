@@ -27,7 +27,7 @@ def lib():
 def declared_functions() -> list[str]:
     text = HEADER.read_text()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(attn_[a-z_]+)\s*\(",
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(attn_[a-z0-9_]+)\s*\(",
                       text, flags=re.M)
 
 
@@ -209,3 +209,37 @@ def test_ring_host_argument_checks(lib):
     n0 = lib.attn_launch_count()
     assert ring() == ATTN_ERR_CUDA
     assert lib.attn_launch_count() == n0
+
+
+def test_debug_exp2_argument_checks(lib):
+    from online_softmax_exact_b200._abi import ATTN_ERR_INVALID_ARG
+
+    assert lib.attn_debug_exp2(None, 2 * A, 16, 1, None) == ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_exp2(A, None, 16, 1, None) == ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_exp2(A, 2 * A, 0, 1, None) == ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_exp2(A, 2 * A, 16, 2, None) == ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_exp2(A, A + 32, 16, 1, None) == ATTN_ERR_INVALID_ARG   # overlap
+    assert lib.attn_debug_exp2(A + 2, 2 * A, 16, 1, None) == ATTN_ERR_INVALID_ARG
+
+
+def test_noalloc_argument_checks(lib):
+    """The allocation-free ring call rejects bad arguments, and sizes its array cannot
+    hold, before any CUDA call."""
+    from online_softmax_exact_b200._abi import (ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED,
+                                                ATTN_NOALLOC_SCRATCH_BYTES)
+
+    def call(B=1, Hq=2, Hkv=2, N=256, d=64, n_chunks=2, q=A):
+        return lib.attn_ring_fwd_host_noalloc(q, 2 * A, 3 * A, 4 * A, 5 * A, B, Hq, Hkv, N, d,
+                                              n_chunks, 1, 0.125, None, None, None)
+
+    assert call(q=None) == ATTN_ERR_INVALID_ARG
+    assert call(Hq=3, Hkv=2) == ATTN_ERR_INVALID_ARG
+    assert call(N=255) == ATTN_ERR_INVALID_ARG           # 2 chunks do not divide 255
+    assert call(d=96) == ATTN_ERR_UNSUPPORTED
+    assert call(n_chunks=64, N=64 * 64) == ATTN_ERR_UNSUPPORTED
+    # Q alone is larger than the array
+    big_n = ATTN_NOALLOC_SCRATCH_BYTES // (2 * 64 * 2) + 256
+    assert call(N=big_n, n_chunks=1) == ATTN_ERR_UNSUPPORTED
+    # a size that fits Q, K, V but not the result and partial slots as well
+    n_fit = ATTN_NOALLOC_SCRATCH_BYTES // (8 * 2 * 64 * 2) * 2
+    assert call(N=n_fit, n_chunks=2) == ATTN_ERR_UNSUPPORTED
