@@ -23,11 +23,12 @@ merges. The line printed by rank 0 reports:
              with the compute chunk by chunk;
   cpu_baseline  the fp64 oracle on the host cores, on a bounded row sample of the
              same workload (rank 0, N=1 only);
-  per_workload  the other workloads at full size (causal_4k, gqa_128k single passes;
-             grid2d_64k_stress as its 4 x 4 grid plus merges and as a single pass), a
-             few device-timed steps each, with the attention kernel's fraction of the
-             burst peak, the merges' GB/s and the oracle's rate on sampled rows
-             (its full-size time extrapolated).
+  per_workload  the other workloads at full size (tiny_chunks4 single pass and as 4
+             partials plus a merge; causal_4k, gqa_128k single passes; grid2d_64k_stress
+             as its 4 x 4 grid plus merges and as a single pass), a few device-timed
+             steps each, with the attention kernel's fraction of the burst peak, the
+             merges' GB/s and the oracle's time: in full for tiny_chunks4 and causal_4k,
+             on sampled rows (full-size time extrapolated) for the others.
 
 With --gpus N > 1 (launched by torchrun), every rank runs its own independent
 problem of the same size (different seed): weak scaling, no data-path collective.
@@ -534,7 +535,8 @@ def run_ours(args, w) -> int:
         del q, k, v, out, ws
         torch.cuda.empty_cache()
         per_workload = run_per_workload(args, dev, peaks, peak_src,
-                                        ["causal_4k", "gqa_128k", "grid2d_64k_stress"])
+                                        ["tiny_chunks4", "causal_4k", "gqa_128k",
+                                         "grid2d_64k_stress"])
 
     total_flops = w.flops * args.steps * world
     value = total_flops / (ms_max * 1e-3) / 1e12
@@ -671,6 +673,28 @@ def run_per_workload(args, dev, peaks: dict, peak_src: str, names: list[str]) ->
                      "inputs larger than L2; no flush",
                "single_pass": {"ms": ms_single, "tflops": tf_single,
                                "frac_of_burst_bf16": tf_single / peak_b}}
+        if w.schedule == "chunks":
+            # KV in n_chunks pieces as partials, then one merge (launch-bound at this size)
+            P, C = w.n_chunks, w.N // w.n_chunks
+            parts = [(torch.empty((B, Hq, N, d), dtype=torch.float32, device=dev),
+                      torch.empty((B, Hq, N), dtype=torch.float32, device=dev))
+                     for _ in range(P)]
+
+            def chunked():
+                for i in range(P):
+                    osx.attn_fwd_partial(q, k, v, q_start=0, q_len=N, kv_start=i * C, kv_len=C,
+                                         causal=w.causal, scale=w.scale, o=parts[i][0],
+                                         lse=parts[i][1], stream=stream)
+                osx.attn_merge([x[0] for x in parts], [x[1] for x in parts], o=o, lse=lse,
+                               stream=stream)
+
+            for _ in range(3):
+                chunked()
+            t_ch = time_reps(chunked, reps, stream, flush)
+            ms_ch = statistics.median(t_ch)
+            rec["chunks_with_merge"] = {
+                "ms": ms_ch, "tflops": w.flops / (ms_ch * 1e-3) / 1e12,
+                "launches": f"{P} attn_fwd_partial + 1 attn_merge per step (launch-bound)"}
         if w.schedule == "grid2d":
             P, C = w.n_chunks, w.N // w.n_chunks
             orders = grid_merge_orders(P, w.seed)
@@ -678,13 +702,13 @@ def run_per_workload(args, dev, peaks: dict, peak_src: str, names: list[str]) ->
                      torch.empty((P, B, Hq, C), dtype=torch.float32, device=dev))
             from online_softmax_exact_b200.schedules import Workspace
 
-            ws = Workspace.for_shape(P, B, Hq, C, d, dev)
+            ws = Workspace.for_shape(P * P, B, Hq, C, d, dev)
             timer = EventTimer(stream)
 
             def grid():
                 grid2d_attention(q, k, v, n_chunks=P, merge_orders=orders, causal=w.causal,
                                  scale=w.scale, out=out_c, workspace=ws, stream=stream,
-                                 timer=timer)
+                                 timer=timer, batched=True)
 
             for _ in range(3):
                 grid()
@@ -708,12 +732,24 @@ def run_per_workload(args, dev, peaks: dict, peak_src: str, names: list[str]) ->
                 "attention_frac_of_burst_bf16": attn_tf / peak_b if attn_tf else None,
                 "merge_gbs": merge_gbs,
                 "merge_frac_of_hbm": merge_gbs / peak_h if merge_gbs else None,
-                "launches": f"{P * P} attn_fwd_partial + {P} attn_merge ({P} parts each, "
-                            "seeded order) per step, one stream"}
+                "launches": f"one attn_fwd_partial_batch launch of the {P * P} cells, then "
+                            f"{P} attn_merge ({P} parts each, seeded order) per step"}
             del ws, out_c
         if osx.attn_device_status() != osx.ATTN_OK:
             raise RuntimeError(f"device-side wait ran out of time in {name}")
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and w.flops <= 2e11:
+            # small enough to time the oracle on the whole workload
+            import oracle
+
+            q_c, k_c, v_c = attention_inputs(w)
+            t0c = time.perf_counter()
+            oracle.attention(q_c, k_c, v_c, causal=w.causal, scale=w.scale)
+            secs = time.perf_counter() - t0c
+            rec["oracle"] = {
+                "tflops": w.flops / secs / 1e12, "full_size_s": secs,
+                "cores": oracle.default_threads(), "rows": B * Hq * N,
+                "note": "fp64 oracle on the whole workload (every row)"}
+        elif not args.no_cpu_baseline:
             r = oracle_sample_throughput(w, args.cpu_seconds_per_workload)
             rec["oracle"] = {
                 "tflops": r["tflops"], "rows_per_s": r["rows"] / r["seconds"],
@@ -763,9 +799,34 @@ def run_e2e(args, w, q_h, k_h, v_h, dev, world) -> dict:
     ms = max_over_ranks(t0.elapsed_time(t1), dev)
     h2d = qp.numel() * 2 + kp.numel() * 2 + vp.numel() * 2
     d2h = o_h.numel() * 4 + l_h.numel() * 4
+
+    # the copies alone, same bytes, same page-locked buffers: what bounds this path
+    def copies(direction):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        if direction == "h2d":
+            for src, dst in ((qp, bufs.q), (kp, bufs.k), (vp, bufs.v)):
+                dst.copy_(src, non_blocking=True)
+        else:
+            o_h.copy_(bufs.o, non_blocking=True)
+            l_h.copy_(bufs.lse, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    copies("h2d")
+    copies("d2h")
+    ms_h2d = min(copies("h2d") for _ in range(3))
+    ms_d2h = min(copies("d2h") for _ in range(3))
     return {"value": w.flops * steps * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
+            "h2d_gbs": h2d / (ms_h2d * 1e-3) / 1e9, "d2h_gbs": d2h / (ms_d2h * 1e-3) / 1e9,
+            "copy_floor_ms": max(ms_h2d, ms_d2h),
+            "copy_floor_note": "each direction's bytes copied alone (page-locked, one stream); "
+                               "the two directions can overlap, so the step cannot be shorter "
+                               "than the slower of them",
             "api": "attn_ring_fwd_host (C ABI; page-locked host buffers; per-chunk copies "
                    "pipelined with the per-query-chunk launches)"}
 

@@ -242,14 +242,52 @@ def ring_attention(q, k, v, *, n_chunks: int, causal: bool, scale: float | None 
     return o_out, l_out
 
 
+def _grid_batched(q, k, v, bounds, merge_orders, causal, scale, o_out, l_out, workspace,
+                  main, timer, fused_merge):
+    """The grid with batched launches: without the fused merge, every cell in one
+    launch, then one merge per query chunk in its order; with it, one launch per merge
+    step s holding cell (i, merge_orders[i][s]) of every query chunk i."""
+    P = len(bounds)
+    if fused_merge:
+        for s_step in range(P):
+            pairs = []
+            for qi in range(P):
+                qs, qe = bounds[qi]
+                ks, ke = bounds[merge_orders[qi][s_step]]
+                pairs.append(dict(q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                                  o=o_out[qi], lse=l_out[qi]))
+            with timer("partial", main):
+                attn_fwd_partial_batch(q, k, v, pairs, causal=causal, scale=scale,
+                                       accumulate=s_step > 0, stream=main)
+        return
+    pairs = []
+    for qi in range(P):
+        qs, qe = bounds[qi]
+        for kv in range(P):
+            ks, ke = bounds[kv]
+            pairs.append(dict(q_start=qs, q_len=qe - qs, kv_start=ks, kv_len=ke - ks,
+                              o=workspace.o[qi * P + kv], lse=workspace.lse[qi * P + kv]))
+    with timer("partial", main):
+        attn_fwd_partial_batch(q, k, v, pairs, causal=causal, scale=scale, stream=main)
+    for qi in range(P):
+        order = merge_orders[qi]
+        with timer("merge", main):
+            attn_merge([workspace.o[qi * P + x] for x in order],
+                       [workspace.lse[qi * P + x] for x in order],
+                       o=o_out[qi], lse=l_out[qi], stream=main)
+
+
 def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], causal: bool,
                      scale: float | None = None, out=None, workspace: Workspace | None = None,
-                     stream=None, timer=None, n_streams: int = 1, fused_merge: bool = False):
+                     stream=None, timer=None, n_streams: int = 1, fused_merge: bool = False,
+                     batched: bool = False):
     """ATTENTION2D's query x key/value grid on one GPU: every (query chunk, key/value
     chunk) cell is a partial attention (fragment-local statistics, section 3); each
     query chunk's partials are merged in the order ``merge_orders[i]`` (any order gives
     the same result, section 2). With ``fused_merge`` the cells of a query chunk are
-    folded into one running accumulator in that order instead. Returns chunk-major
+    folded into one running accumulator in that order instead. With ``batched`` the
+    cells go through ``attn_fwd_partial_batch`` (all n_chunks^2 cells in one launch, at
+    most 48; with ``fused_merge``, one launch per merge step). Returns chunk-major
     (O, LSE).
     """
     timer = timer or _NO_TIMER
@@ -257,6 +295,20 @@ def grid2d_attention(q, k, v, *, n_chunks: int, merge_orders: list[list[int]], c
     bounds = chunk_bounds(N, n_chunks)
     C = N // n_chunks
     o_out, l_out = _alloc_out(q, n_chunks, out)
+    for qi in range(n_chunks):
+        if sorted(merge_orders[qi]) != list(range(n_chunks)):
+            raise ValueError("each merge order must be a permutation of the chunk indices")
+    if batched:
+        if n_chunks * n_chunks > 48 and not fused_merge:
+            raise ValueError("a batched grid holds at most 48 cells per launch")
+        need = n_chunks * n_chunks
+        if not fused_merge and (workspace is None or workspace.o.shape[0] < need
+                                or workspace.o.shape[1:] != (B, Hq, C, d)):
+            workspace = Workspace.for_shape(need, B, Hq, C, d, q.device)
+        main = stream if stream is not None else torch.cuda.current_stream(q.device)
+        _grid_batched(q, k, v, bounds, merge_orders, causal, scale, o_out, l_out, workspace,
+                      main, timer, fused_merge)
+        return o_out, l_out
     n_streams = max(1, min(n_streams, n_chunks))
     need = n_chunks * n_streams
     if not fused_merge and (workspace is None or workspace.o.shape[0] < need

@@ -78,10 +78,14 @@ def test_grid2d_64k_stress(osx):
     w = get("grid2d_64k_stress")
     q, k, v = attention_inputs(w)
     qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
-    for fused in (False, True):
-        oc, lc = grid2d_attention(qg, kg, vg, n_chunks=w.n_chunks,
-                                  merge_orders=grid_merge_orders(w.n_chunks, w.seed),
-                                  causal=w.causal, scale=w.scale, fused_merge=fused)
-        assert osx.attn_device_status() == osx.ATTN_OK
-        o, lse = chunks_to_sequence(oc, lc)
-        check_sampled(o, lse, q, k, v, w, 96 if not fused else 48)
+    # per-cell launches and the batched launch the benchmark times, each with partial
+    # buffers and merges and with the fused running merge
+    for batched in (False, True):
+        for fused in (False, True):
+            oc, lc = grid2d_attention(qg, kg, vg, n_chunks=w.n_chunks,
+                                      merge_orders=grid_merge_orders(w.n_chunks, w.seed),
+                                      causal=w.causal, scale=w.scale, fused_merge=fused,
+                                      batched=batched)
+            assert osx.attn_device_status() == osx.ATTN_OK
+            o, lse = chunks_to_sequence(oc, lc)
+            check_sampled(o, lse, q, k, v, w, 96 if batched and not fused else 32)
