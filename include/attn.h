@@ -304,9 +304,10 @@ attn_status_t attn_debug_wait_timeout(int64_t limit_cycles, void* stream);
  * attn_debug_exp2 - check of the two exponentials the softmax uses, for tests:
  * y[i] = 2^x[i] through the FMA-pipe polynomial (use_poly = 1: Cody and Waite's
  * reduction to x = n + f, |f| <= 1/2, and a degree-3 minimax polynomial for 2^f, max
- * relative error 7.5e-5 for -126 <= x <= 127) or through the exp unit's ex2.approx
- * (use_poly = 0). The polynomial clamps x below at -126 (it gives at most 2^-125 there,
- * not 0). x, y: device fp32 arrays of n >= 1 values, not overlapping.
+ * relative error 7.5e-5 for -125.5 <= x <= 127; just above -126 the result can come
+ * out denormal, off by at most 2^-138 in absolute terms) or through the exp unit's
+ * ex2.approx (use_poly = 0). The polynomial clamps x below at -126 (it gives at most
+ * 2^-125 there, not 0). x, y: device fp32 arrays of n >= 1 values, not overlapping.
  */
 attn_status_t attn_debug_exp2(const float* x, float* y, int64_t n, int use_poly, void* stream);
 

@@ -5,8 +5,10 @@ Method (the kernel's own): Cody and Waite's reduction x = n + f with n = round(x
 |f| <= 1/2, a degree-3 polynomial for 2^f fitted by the Remez exchange algorithm for
 minimax relative error (csrc/exp2_poly_fit.py: 7.48e-5 after rounding the coefficients
 to fp32), and n added to the exponent field. Bound checked here: relative error <=
-7.48e-5 plus a few fp32 roundings (2^-22) against 2^x in fp64; inputs below -126 give
-a value in [0, 2^-125].
+7.48e-5 plus a few fp32 roundings (2^-22) against 2^x in fp64 for x >= -125.5. Just
+above -126 (n = -126) the polynomial's value below 1 makes the result denormal: the
+error there is checked in absolute terms (<= 2^-138). Inputs below -126 give a value in
+[0, 2^-125].
 """
 
 from __future__ import annotations
@@ -44,11 +46,14 @@ def test_poly_within_its_bound_of_the_exact_value(osx):
     x = _xs()
     y = osx.attn_debug_exp2(x.cuda(), use_poly=True).cpu().double()
     exact = torch.exp2(x.double())
-    rel = ((y - exact) / exact).abs()
     assert torch.isfinite(y).all()
+    normal = x >= -125.5
+    rel = ((y[normal] - exact[normal]) / exact[normal]).abs()
     worst = float(rel.max())
     print(f"polynomial 2^x: max relative error {worst:.3e} (bound {POLY_REL:.3e})")
     assert worst <= POLY_REL
+    # n = -126: the result may be denormal, absolutely tiny errors only
+    assert float((y[~normal] - exact[~normal]).abs().max()) <= 2.0 ** -138
 
 
 def test_poly_against_the_exp_unit(osx):
