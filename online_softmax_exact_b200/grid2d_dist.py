@@ -30,7 +30,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import attn_fwd_partial, attn_merge
+from . import ATTN_OK, AttnError, attn_device_status, attn_fwd_partial, attn_merge
 
 
 def grid_coords(rank: int, p_q: int, p_kv: int) -> tuple[int, int]:
@@ -125,7 +125,7 @@ class _Exchange:
 def grid2d_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, p_q: int,
                           p_kv: int, causal: bool, scale: float | None = None,
                           row_group=None, merge_order=None, partial=None, merge=None,
-                          overlap: bool = False, n_splits: int = 2):
+                          overlap: bool = False, n_splits: int = 2, check_status: bool = True):
     """This rank's fragment of the grid, then the reduce-scatter along its row.
 
     q: [B, Hq, Cq, d], query chunk i of the sequence (rows i*Cq ..); k, v:
@@ -142,7 +142,9 @@ def grid2d_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, 
 
     ``partial(q, k, v, *, q_off, kv_off, causal, scale) -> (O, LSE)`` and
     ``merge(o_parts, lse_parts) -> (O, LSE)`` replace the local compute; ``merge``
-    gets parts of shape [R, B, H, d] / [R, B, H].
+    gets parts of shape [R, B, H, d] / [R, B, H]. With the library's own compute and
+    ``check_status``, the call ends by synchronising the current stream and raising
+    ``AttnError`` if a kernel recorded a device-side time-out.
     """
     rank = dist.get_rank()
     if dist.get_world_size() != p_q * p_kv:
@@ -152,13 +154,16 @@ def grid2d_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, 
     Hkv, Ckv = k.shape[1], k.shape[2]
     if scale is None:
         scale = d ** -0.5
+    library = partial is None and merge is None
     partial = partial or _default_partial
     merge = merge or _default_merge
     order = list(range(p_kv)) if merge_order is None else list(merge_order)
     if sorted(order) != list(range(p_kv)):
         raise ValueError("merge_order must be a permutation of the key/value chunks")
     if p_kv == 1:
-        return partial(q, k, v, q_off=i * Cq, kv_off=j * Ckv, causal=causal, scale=scale)
+        res = partial(q, k, v, q_off=i * Cq, kv_off=j * Ckv, causal=causal, scale=scale)
+        _check(library and check_status)
+        return res
     if Cq < p_kv:
         raise ValueError("a query chunk needs at least one row per column of the grid")
     slices = row_slices(Cq, p_kv)
@@ -174,6 +179,14 @@ def grid2d_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, 
         pending.append(_Exchange(o, lse, slices, j, row_group, order, merge,
                                  async_op=overlap))
     parts = [x.merged() for x in pending]
+    _check(library and check_status)
     if len(parts) == 1:
         return parts[0]
     return torch.cat([p[0] for p in parts], dim=1), torch.cat([p[1] for p in parts], dim=1)
+
+
+def _check(enabled: bool) -> None:
+    if enabled:
+        st = attn_device_status()
+        if st != ATTN_OK:
+            raise AttnError(st, "grid2d_attention_dist")

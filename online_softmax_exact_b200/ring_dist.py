@@ -31,7 +31,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import attn_fwd_partial, attn_fwd_partial_acc
+from . import ATTN_OK, AttnError, attn_device_status, attn_fwd_partial, attn_fwd_partial_acc
 
 
 def ring_steps(rank: int, world: int, causal: bool) -> list[tuple[int, int, bool]]:
@@ -103,7 +103,7 @@ def _peers(group, rank, world):
 
 def ring_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
                         scale: float | None = None, group=None, out=None, fold=None,
-                        layout: str = "contiguous"):
+                        layout: str = "contiguous", check_status: bool = True):
     """This rank's query chunk attends every rank's key/value chunk, in ring order.
 
     q: [B, Hq, C, d]; k, v: [B, Hkv, C, d] - this rank's chunk of the sequence (global
@@ -117,7 +117,9 @@ def ring_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, ca
     local compute (default: the library's partial attention on the current stream):
     it folds keys k/v (global positions from kv_off) into the accumulator (o, lse) of
     queries q (positions from q_off); ``first`` says that the accumulator holds
-    nothing yet.
+    nothing yet. With the default fold and ``check_status``, the call ends by
+    synchronising the current stream and raising ``AttnError`` if a kernel recorded a
+    device-side time-out (its results would be unspecified).
     """
     if layout not in ("contiguous", "zigzag"):
         raise ValueError("layout must be 'contiguous' or 'zigzag'")
@@ -130,6 +132,7 @@ def ring_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, ca
         raise ValueError("the zigzag layout needs an even chunk length")
     if scale is None:
         scale = d ** -0.5
+    library_fold = fold is None
     fold = fold or _default_fold
     if out is None:
         o = torch.empty((B, Hq, C, d), dtype=torch.float32, device=q.device)
@@ -143,7 +146,15 @@ def ring_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, ca
     else:
         _ring_zigzag(q, k, v, o, lse, rank, world, causal, scale, fold, nxt_rank,
                      prv_rank, group)
+    if library_fold and check_status:
+        _raise_on_device_failure("ring_attention_dist")
     return o, lse
+
+
+def _raise_on_device_failure(where: str) -> None:
+    st = attn_device_status()
+    if st != ATTN_OK:
+        raise AttnError(st, where)
 
 
 def _exchange(cur, nxt, nxt_rank, prv_rank, group):

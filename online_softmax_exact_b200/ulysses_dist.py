@@ -13,7 +13,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import attn_fwd
+from . import ATTN_OK, AttnError, attn_device_status, attn_fwd
 
 
 def _default_attend(q, k, v, *, causal, scale):
@@ -46,14 +46,15 @@ def _heads_to_seq(x: torch.Tensor, world: int, group) -> torch.Tensor:
 
 def ulysses_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
                            causal: bool, scale: float | None = None, group=None,
-                           attend=None):
+                           attend=None, check_status: bool = True):
     """q: [B, Hq, C, d]; k, v: [B, Hkv, C, d] - chunk ``rank`` of the sequence on every
     rank of ``group`` (P ranks; Hq and Hkv divisible by P, and Hq/Hkv groups stay
     whole since head g of q reads head g // (Hq/Hkv) of k). Returns this rank's chunk
     of (O [B, Hq, C, d], LSE [B, Hq, C]) in fp32.
 
     ``attend(q, k, v, *, causal, scale) -> (O, LSE)`` replaces the local attention
-    (default: the library's single pass).
+    (default: the library's single pass; with ``check_status`` its device status is
+    checked after it, raising ``AttnError`` on a device-side time-out).
     """
     world = dist.get_world_size(group)
     B, Hq, C, d = q.shape
@@ -62,9 +63,14 @@ def ulysses_attention_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
         raise ValueError("the head counts must divide among the ranks")
     if scale is None:
         scale = d ** -0.5
+    library = attend is None
     attend = attend or _default_attend
     qh = _seq_to_heads(q, world, group)
     kh = _seq_to_heads(k, world, group)
     vh = _seq_to_heads(v, world, group)
     o, lse = attend(qh, kh, vh, causal=causal, scale=scale)
+    if library and check_status:
+        st = attn_device_status()
+        if st != ATTN_OK:
+            raise AttnError(st, "ulysses_attention_dist")
     return _heads_to_seq(o, world, group), _heads_to_seq(lse, world, group)
