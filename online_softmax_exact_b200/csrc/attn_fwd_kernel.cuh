@@ -97,6 +97,12 @@ struct FwdParams {
 #define OSX_EMU_MASK_128 0x0000u
 #endif
 
+#ifndef OSX_STAGES_64
+#define OSX_STAGES_64 3
+#endif
+#ifndef OSX_KSTAGES_128
+#define OSX_KSTAGES_128 2
+#endif
 #ifndef OSX_ROW_REGS_SOFTMAX
 #define OSX_ROW_REGS_SOFTMAX 216
 #endif
@@ -114,15 +120,17 @@ template <int D, bool kRow = false>
 struct FwdCfg {
   static constexpr int kBM = 128;                    // rows per Q tile
   static constexpr int kBN = 128;                    // keys per KV tile
-  static constexpr int kStages = (D == 128) ? 2 : 3; // K and V ring depth
+  // K and V ring depths (K is needed a P.V earlier than V)
+  static constexpr int kKStages = (D == 128) ? OSX_KSTAGES_128 : OSX_STAGES_64;
+  static constexpr int kVStages = (D == 128) ? 2 : OSX_STAGES_64;
   static constexpr uint32_t kTileBytes = kBM * D * 2;  // one 128-row bf16 tile
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = 2 * kTileBytes;
-  static constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
-  static constexpr uint32_t kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr uint32_t kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr uint32_t kBarOff = kVOff + kVStages * kTileBytes;
   // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S],
   // s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 2 + 4 * kStages + 6 + 1;
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 6 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   // half-row exchange (two threads per row only): maxima [tile][parity][half][row],
   // denominators [tile][half][row]
@@ -291,11 +299,13 @@ __device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP,
 }
 
 // One thread per row: 32 of the row's scores -> 16 columns of bf16 P pairs at tP, against
-// a known maximum (x = S * c - m: NM2 holds -m twice); returns the sum of the 32 values
-// of P. Masked elements (index > climit) get x = -inf, for which ex2 gives exactly 0.
+// a known maximum (x = S * c - m); returns the sum of the 32 values of P. Masked elements
+// (index > climit) get x = -inf, for which ex2 gives exactly 0.
 template <bool kMasked, uint32_t kEmu>
-__device__ __forceinline__ float softmax_row32(const uint32_t (&s)[32], uint32_t tP,
-                                               uint64_t C2, uint64_t NM2, int climit) {
+__device__ __forceinline__ float softmax_row32(const uint32_t (&s)[32], uint32_t tP, float c,
+                                               float m_use, int climit) {
+  const uint64_t C2 = f2_pack(c, c);
+  const uint64_t NM2 = f2_pack(-m_use, -m_use);
   uint64_t A01 = 0, A23 = 0;
   uint32_t pk[16];
 #pragma unroll
@@ -347,9 +357,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int B_QF = 0, B_QE = 1;
-  const int B_KF = 2, B_KE = 2 + C::kStages, B_VF = 2 + 2 * C::kStages,
-            B_VE = 2 + 3 * C::kStages;
-  const int B_SF = 2 + 4 * C::kStages, B_PF = B_SF + 2, B_OD = B_SF + 4, B_DRAIN = B_SF + 6;
+  const int B_KF = 2, B_KE = 2 + C::kKStages, B_VF = 2 + 2 * C::kKStages,
+            B_VE = 2 + 2 * C::kKStages + C::kVStages;
+  const int B_SF = 2 + 2 * C::kKStages + 2 * C::kVStages, B_PF = B_SF + 2, B_OD = B_SF + 4,
+            B_DRAIN = B_SF + 6;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -357,9 +368,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     *abort_flag = 0;
     mbar_init(bar(B_QF), 1);
     mbar_init(bar(B_QE), 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(bar(B_KF + s), 1);
       mbar_init(bar(B_KE + s), 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(bar(B_VF + s), 1);
       mbar_init(bar(B_VE + s), 1);
     }
@@ -432,14 +445,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               tma_load_3d(sbase + C::kKOff + ks * C::kTileBytes + h * 16384, &tmK, bar(B_KF + ks),
                           h * 64, pr.kv_row0 + j * 128, kvh);
             ++k_arms;
-            if (++ks == C::kStages) { ks = 0; kph ^= 1; }
+            if (++ks == C::kKStages) { ks = 0; kph ^= 1; }
             if (!(ok = mbar_wait(bar(B_VE + vs), vph ^ 1, abort_flag, p.status))) break;
             mbar_arrive_expect_tx(bar(B_VF + vs), C::kTileBytes);
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sbase + C::kVOff + vs * C::kTileBytes + h * 16384, &tmV, bar(B_VF + vs),
                           h * 64, pr.kv_row0 + j * 128, kvh);
             ++v_arms;
-            if (++vs == C::kStages) { vs = 0; vph ^= 1; }
+            if (++vs == C::kVStages) { vs = 0; vph ^= 1; }
           }
         }
         // Wait until every copy issued has landed (the last armed phase of each full
@@ -448,10 +461,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // flight. Bounded; if it runs out, wait a fixed time instead.
         bool drained = true;
         if (qcount > 0) drained &= mbar_wait_drain(bar(B_QF), (qcount - 1) & 1, kDrainLimitNs);
-        for (int st = 0; st < C::kStages; ++st) {
-          const int kn = k_arms / C::kStages + (st < k_arms % C::kStages ? 1 : 0);
-          const int vn = v_arms / C::kStages + (st < v_arms % C::kStages ? 1 : 0);
+        for (int st = 0; st < C::kKStages; ++st) {
+          const int kn = k_arms / C::kKStages + (st < k_arms % C::kKStages ? 1 : 0);
           if (kn > 0) drained &= mbar_wait_drain(bar(B_KF + st), (kn - 1) & 1, kDrainLimitNs);
+        }
+        for (int st = 0; st < C::kVStages; ++st) {
+          const int vn = v_arms / C::kVStages + (st < v_arms % C::kVStages ? 1 : 0);
           if (vn > 0) drained &= mbar_wait_drain(bar(B_VF + st), (vn - 1) & 1, kDrainLimitNs);
         }
         if (!drained) {
@@ -528,7 +543,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (t == 1) {
                   ++pv_steps;
                   mma_commit(bar(B_VE + vs));
-                  if (++vs == C::kStages) { vs = 0; vph ^= 1; }
+                  if (++vs == C::kVStages) { vs = 0; vph ^= 1; }
                 }
               }
               issue_qk(t, ks);
@@ -536,7 +551,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
             if (!ok) break;
             mma_commit(bar(B_KE + ks));
-            if (++ks == C::kStages) { ks = 0; kph ^= 1; }
+            if (++ks == C::kKStages) { ks = 0; kph ^= 1; }
           }
           if (!ok) break;
           mma_commit(bar(B_QE));
@@ -552,7 +567,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (!ok) break;
           ++pv_steps;
           mma_commit(bar(B_VE + vs));
-          if (++vs == C::kStages) { vs = 0; vph ^= 1; }
+          if (++vs == C::kVStages) { vs = 0; vph ^= 1; }
         }
       }
     }
@@ -671,12 +686,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 sum = softmax_half<false, false, C::kEmu>(s, tS, c, m_new, climit, nullptr);
               } else {
                 const uint32_t a2 = pack_bf16x2(alpha, alpha);
-  #pragma unroll 1
+#pragma unroll 1
                 for (int q2 = 0; q2 < 2; ++q2) {  // rare: kept small rather than fast
                   uint32_t pv[16];
                   tmem_ld16(tS + q2 * 16, pv);
                   tmem_ld_wait(pv);
-  #pragma unroll
+#pragma unroll
                   for (int i = 0; i < 16; ++i) pv[i] = mul_bf16x2(pv[i], a2);
                   tmem_st16(tS + q2 * 16, pv);
                 }
@@ -687,7 +702,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             float mx = -INFINITY;
             {
               float m0 = -INFINITY, m1 = -INFINITY;
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float v0 = (2 * i > climit) ? -INFINITY : __uint_as_float(s[0][2 * i]);
                 const float v1 = (2 * i + 1 > climit) ? -INFINITY : __uint_as_float(s[0][2 * i + 1]);
@@ -716,12 +731,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const bool moved = (m_new != m) && (j > 0);
           if (__any_sync(0xffffffffu, moved)) {
             const float a = moved ? alpha : 1.f;
-  #pragma unroll
+#pragma unroll
             for (int q4 = 0; q4 < D / 64; ++q4) {
               uint32_t ov[32];
               tmem_ld32(tO + q4 * 32, ov);
               tmem_ld_wait(ov);
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * a);
               tmem_st32(tO + q4 * 32, ov);
             }
@@ -773,7 +788,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             lse_out = M + lg * 0.69314718055994530942f;
           }
         }
-  #pragma unroll
+#pragma unroll
         for (int q4 = 0; q4 < D / 64; ++q4) {
           uint32_t ov[32];
           tmem_ld32(tO + q4 * 32, ov);
@@ -781,10 +796,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (row_valid) {
             float* dst = orow_of() + q4 * 32;
             float res[32];
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
             if (a != 0.f) {  // only then is the old accumulator read
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 32; i += 4) {
                 const float4 old = *reinterpret_cast<const float4*>(dst + i);
                 res[i] = fmaf(a, old.x, res[i]);
@@ -794,14 +809,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               }
             }
             if (p.o_vec8) {
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 4; ++i)
                 st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
                              res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
                              res[8 * i + 7]);
             } else {
               float4* o4 = reinterpret_cast<float4*>(dst);
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 8; ++i)
                 o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
             }
@@ -822,7 +837,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0);
       const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0);
       const float c = p.scale_log2;
-      const uint64_t C2 = f2_pack(c, c);
       int scount = 0, ocount = 0;
       bool ok = true;
 
@@ -869,7 +883,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
 
           uint32_t s[4][32];
-  #pragma unroll
+#pragma unroll
           for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, s[q]);
           tmem_ld_wait(s[0]);
           reg_fence(s[1]);
@@ -881,20 +895,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int cl = lim_row - j * 128;  // keys with local index <= climit are visible
           const int climit = cl < -1 ? -1 : (cl > 127 ? 127 : cl);
 
-          // tile maximum of the raw scores over the visible keys (four partial maxima)
+          // tile maximum of the raw scores over the visible keys (four partial maxima);
+          // two separate loops, so that unmasked tiles carry no per-element selects
           float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  #pragma unroll
-          for (int q = 0; q < 4; ++q)
-  #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float v0 = __uint_as_float(s[q][2 * i]), v1 = __uint_as_float(s[q][2 * i + 1]);
-              if (need_mask) {
-                v0 = (32 * q + 2 * i > climit) ? -INFINITY : v0;
-                v1 = (32 * q + 2 * i + 1 > climit) ? -INFINITY : v1;
+          if (need_mask) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float v0 =
+                    (32 * q + 2 * i > climit) ? -INFINITY : __uint_as_float(s[q][2 * i]);
+                const float v1 =
+                    (32 * q + 2 * i + 1 > climit) ? -INFINITY : __uint_as_float(s[q][2 * i + 1]);
+                float& acc = mxa[(q & 1) * 2 + (i & 1)];
+                acc = fmax3(acc, v0, v1);
               }
-              float& acc = mxa[(q & 1) * 2 + (i & 1)];
-              acc = fmax3(acc, v0, v1);
-            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float& acc = mxa[(q & 1) * 2 + (i & 1)];
+                acc = fmax3(acc, __uint_as_float(s[q][2 * i]), __uint_as_float(s[q][2 * i + 1]));
+              }
+          }
           const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
           // The exponent base moves only when the tile maximum exceeds it by more than 8
           // (log2 units), and then to the tile maximum: numerator and denominator share the
@@ -904,21 +928,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // 1 when unchanged (also when both are -inf), 0 when m was -inf
           const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
           const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          const uint64_t NM2 = f2_pack(-m_use, -m_use);
 
           // P over S's first 64 columns (32 keys -> 16 columns): every score is in
           // registers already
           float sum;
           if (need_mask) {
-            sum = softmax_row32<true, 0u>(s[0], tS, C2, NM2, climit);
-            sum += softmax_row32<true, 0u>(s[1], tS + 16, C2, NM2, climit - 32);
-            sum += softmax_row32<true, 0u>(s[2], tS + 32, C2, NM2, climit - 64);
-            sum += softmax_row32<true, 0u>(s[3], tS + 48, C2, NM2, climit - 96);
+            sum = softmax_row32<true, 0u>(s[0], tS, c, m_use, climit);
+            sum += softmax_row32<true, 0u>(s[1], tS + 16, c, m_use, climit - 32);
+            sum += softmax_row32<true, 0u>(s[2], tS + 32, c, m_use, climit - 64);
+            sum += softmax_row32<true, 0u>(s[3], tS + 48, c, m_use, climit - 96);
           } else {
-            sum = softmax_row32<false, C::kEmu>(s[0], tS, C2, NM2, 127);
-            sum += softmax_row32<false, C::kEmu>(s[1], tS + 16, C2, NM2, 127);
-            sum += softmax_row32<false, C::kEmu>(s[2], tS + 32, C2, NM2, 127);
-            sum += softmax_row32<false, C::kEmu>(s[3], tS + 48, C2, NM2, 127);
+            sum = softmax_row32<false, C::kEmu>(s[0], tS, c, m_use, 127);
+            sum += softmax_row32<false, C::kEmu>(s[1], tS + 16, c, m_use, 127);
+            sum += softmax_row32<false, C::kEmu>(s[2], tS + 32, c, m_use, 127);
+            sum += softmax_row32<false, C::kEmu>(s[3], tS + 48, c, m_use, 127);
           }
           l = l * alpha + sum;
 
@@ -927,12 +950,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const bool moved = (m_new != m) && (j > 0);
           if (__any_sync(0xffffffffu, moved)) {
             const float a = moved ? alpha : 1.f;
-  #pragma unroll 1
+#pragma unroll 1
             for (int q4 = 0; q4 < D / 32; ++q4) {
               uint32_t ov[32];
               tmem_ld32(tO + q4 * 32, ov);
               tmem_ld_wait(ov);
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * a);
               tmem_st32(tO + q4 * 32, ov);
             }
@@ -979,7 +1002,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             lse_out = M + lg * 0.69314718055994530942f;
           }
         }
-  #pragma unroll 1
+#pragma unroll 1
         for (int q4 = 0; q4 < D / 32; ++q4) {
           uint32_t ov[32];
           tmem_ld32(tO + q4 * 32, ov);
@@ -987,10 +1010,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (row_valid) {
             float* dst = orow_of() + q4 * 32;
             float res[32];
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
             if (a != 0.f) {  // only then is the old accumulator read
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 32; i += 4) {
                 const float4 old = *reinterpret_cast<const float4*>(dst + i);
                 res[i] = fmaf(a, old.x, res[i]);
@@ -1000,14 +1023,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               }
             }
             if (p.o_vec8) {
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 4; ++i)
                 st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
                              res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
                              res[8 * i + 7]);
             } else {
               float4* o4 = reinterpret_cast<float4*>(dst);
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 8; ++i)
                 o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
             }
