@@ -111,8 +111,8 @@ def load_peaks() -> tuple[dict, str]:
 # digest of the kernel sources the capture ran, and by launch mode; any other source
 # gives null.
 MEASURED_TRAFFIC: dict[str, dict[str, float]] = {
-    "a752dd82299434a69f27bb3fa971ffecc73ec1aaddcbc79fa2fb5ab44709cdcf":
-        {"batched": 3_945_757_696 + 2_406_406_400},
+    "65af274ce483d8fbdfa0e65d8ea0b5414450d0570c95c31f32f2913ff4837d1e":
+        {"batched": 3_588_927_744 + 2_407_559_424},
 }
 
 
