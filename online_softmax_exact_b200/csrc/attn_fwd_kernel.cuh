@@ -12,31 +12,26 @@
 //     one (query chunk, key/value chunk) pair, held as two 128-row tiles in ping-pong:
 //     the tensor core works on one tile while the other tile's softmax runs; a launch
 //     carries up to kMaxPairs pairs, their units in one static schedule;
-//   * warp 16 issues TMA loads (Q tiles once per unit, K and V tiles through a ring of
+//   * warp 8 issues TMA loads (Q tiles once per unit, K and V tiles through rings of
 //     shared-memory stages, 128-byte swizzle);
-//   * warp 17 owns tensor memory and issues tcgen05.mma from one thread:
+//   * warp 9 owns tensor memory and issues tcgen05.mma from one thread:
 //     S_t = Q_t K_j^T (both operands in shared memory) into TMEM, then O_t += P_t V_j
 //     with P_t read from TMEM (written there by the softmax warps over S_t's columns);
-//   * four softmax warpgroups: warpgroup 2t + h handles key half h (64 of the 128 keys of
-//     a tile) of every row of tile t, one row per thread (TMEM lane = row), so each
-//     row's softmax is split over two threads that exchange their half-row maxima (and
-//     at the end their half denominators) through shared memory under a 64-thread
-//     named barrier. A thread reads its 64 scores with tcgen05.ld, exponentiates with
-//     ex2, sums, packs P to bf16 and writes it back with tcgen05.st. The exponent base
-//     is the running maximum m, moved only when a tile maximum exceeds it by more than
-//     8 (log2 units); exactness is kept because numerator and denominator share the
-//     same base. In the common case the exponentials are computed against the current
-//     m while the tile maximum is reduced alongside; if m moves, it moves by a whole
-//     number of octaves, so the P already written is rescaled by an exact power of two
-//     (recomputed only after a jump so large that it may have overflowed), and the
-//     threads rescale their halves of O in TMEM;
+//   * two softmax warpgroups: warpgroup t owns Q tile t, one thread per query row (TMEM
+//     lane = row), all 128 keys of each key tile. A thread reads its 128 scores with
+//     tcgen05.ld, reduces the tile maximum, and only then exponentiates (ex2, and at
+//     d = 64 part of the values through an FMA-pipe polynomial), sums, packs P to bf16
+//     and writes it back with tcgen05.st. The exponent base is the running maximum m,
+//     moved only when a tile maximum exceeds it by more than 8 (log2 units); exactness
+//     is kept because numerator and denominator share the same base. When m moves, the
+//     thread rescales its row of O in TMEM before releasing P;
 //   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32; in accumulate mode
 //     the result is first combined with the normalised partial (O_acc, LSE_acc) already
 //     in o/lse by the log-sum-exp rule of the merge (weights e^(LSE - max LSE)).
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [384,384+D). Half h of P_t (bf16 pairs) overwrites S_t columns [64h, 64h+32),
-// inside that half's own score columns.
+// O_1 [384,384+D). P_t (bf16 pairs, keys in order) overwrites S_t columns [0,64): a
+// thread holds all its scores in registers before it stores any P.
 //
 // Keys of the parent that lie past a pair's chunk but inside the tensor maps (pairs of a
 // batched launch) are read into the pair's last key tile. Their scores are masked, so
@@ -86,37 +81,25 @@ struct FwdParams {
 
 // Pairs (bit i: pair i of every 16) of a thread's scores whose 2^x comes from the FMA
 // pipe in unmasked tiles, per head dimension. Measured on B200 (attn_fwd, TFLOP/s): at
-// D = 64, 2 pairs of 16 (12.5%) gain ~2% on large-logit inputs and ~1% on N(0,1); 4
-// pairs or more lose (the softmax is latency- and issue-bound, not exp-unit-bound, and
-// each polynomial costs ~5 instructions per value against 1). At D = 128 any share
-// loses 1-5%.
+// D = 64, 4 pairs of 16 (25%) gain 1-2% over none; at D = 128 any share loses (the
+// polynomial's ~5 instructions per value, against 1, compete for issue slots with a
+// softmax that shares its tile period with twice the tensor work).
 #ifndef OSX_EMU_MASK_64
-#define OSX_EMU_MASK_64 0x0202u
+#define OSX_EMU_MASK_64 0x2222u
 #endif
 #ifndef OSX_EMU_MASK_128
 #define OSX_EMU_MASK_128 0x0000u
 #endif
-
+// K and V ring depths: 3 + 3 stages at D = 64; 2 + 2 at D = 128 (a third K stage fits in
+// shared memory but measured no gain)
 #ifndef OSX_STAGES_64
 #define OSX_STAGES_64 3
 #endif
 #ifndef OSX_KSTAGES_128
 #define OSX_KSTAGES_128 2
 #endif
-#ifndef OSX_ROW_REGS_SOFTMAX
-#define OSX_ROW_REGS_SOFTMAX 216
-#endif
-#ifndef OSX_ROW_EMU_MASK_64
-#define OSX_ROW_EMU_MASK_64 0x2222u
-#endif
-#ifndef OSX_ROW_EMU_MASK_128
-#define OSX_ROW_EMU_MASK_128 0x0000u
-#endif
 
-// kRow selects the softmax layout: false, two threads per query row (each with 64 of a
-// tile's 128 keys; four softmax warpgroups, 640 threads); true, one thread per row (all
-// 128 keys; two softmax warpgroups, 384 threads, more registers per thread).
-template <int D, bool kRow = false>
+template <int D>
 struct FwdCfg {
   static constexpr int kBM = 128;                    // rows per Q tile
   static constexpr int kBN = 128;                    // keys per KV tile
@@ -132,30 +115,23 @@ struct FwdCfg {
   // s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 6 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
-  // half-row exchange (two threads per row only): maxima [tile][parity][half][row],
-  // denominators [tile][half][row]
-  static constexpr uint32_t kXchOff = (kMiscOff + 16 + 127) & ~127u;
-  static constexpr uint32_t kXlOff = kXchOff + 2 * 2 * 2 * 128 * 4;
-  static constexpr uint32_t kSmemBytes =
-      (kRow ? kXchOff : kXlOff + 2 * 2 * 128 * 4) + 1024;  // + alignment slack
-  // two threads per row: warpgroups 0-3 softmax (tile t = wg / 2, key half h = wg % 2),
-  // warpgroup 4 {TMA producer, MMA issuer, 2 idle}; one thread per row: warpgroups 0-1
-  // softmax (tile t = wg), warpgroup 2 {producer, MMA issuer, 2 idle}
-  static constexpr int kThreads = kRow ? 384 : 640;
-  static constexpr int kSoftmaxWarps = kRow ? 8 : 16;
-  static constexpr int kWarpProducer = kSoftmaxWarps, kWarpMma = kSoftmaxWarps + 1;
+  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  // warpgroups 0-1: softmax (tile t = warpgroup); warpgroup 2: {TMA producer, MMA
+  // issuer, 2 idle}
+  static constexpr int kThreads = 384;
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr int kWarpProducer = 8, kWarpMma = 9;
   // arrivals on a tile's p_full barrier: one per softmax warp of the tile
-  static constexpr int kPFullCount = kRow ? 4 : 8;
-  // Registers per thread. Each SM sub-partition hosts one warp of each warpgroup, so the
-  // warpgroups' shares add up to at most 512 per lane (the sub-partition's 16K registers)
-  // and to the launch's total: two threads per row, 96 at launch, softmax 104, the rest
-  // 64 (4 * 104 + 64 = 5 * 96); one thread per row, 168 at launch, softmax 216, the rest
-  // 72 (2 * 216 + 72 = 3 * 168).
-  static constexpr int kRegsSoftmax = kRow ? OSX_ROW_REGS_SOFTMAX : 104;
-  static constexpr int kRegsOther = kRow ? 504 - 2 * OSX_ROW_REGS_SOFTMAX : 64;
+  static constexpr int kPFullCount = 4;
+  // Registers per thread: 168 at launch (65536 / 384, rounded down to a multiple of 8);
+  // after setmaxnreg the softmax warpgroups hold 216 and warpgroup 2 holds 72
+  // (2 * 216 + 72 = 3 * 168, the launch's total: each SM sub-partition hosts one warp of
+  // each warpgroup, so its 16K registers bound the sum). A softmax thread holds its
+  // row's 128 scores in registers.
+  static constexpr int kRegsSoftmax = 216;
+  static constexpr int kRegsOther = 72;
   // pairs of each 32-score block whose 2^x comes from the FMA pipe (bit i: pair i)
-  static constexpr uint32_t kEmu = kRow ? ((D == 64) ? OSX_ROW_EMU_MASK_64 : OSX_ROW_EMU_MASK_128)
-                                        : ((D == 64) ? OSX_EMU_MASK_64 : OSX_EMU_MASK_128);
+  static constexpr uint32_t kEmu = (D == 64) ? OSX_EMU_MASK_64 : OSX_EMU_MASK_128;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 };
 
@@ -241,63 +217,6 @@ __device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0) {
   fence_proxy_async_smem();
 }
 
-// One thread's half row of P for one 128-key tile (64 scores in s): x = S * c - m
-// (packed pairs), P = 2^x, written to TMEM as 32 columns of bf16 pairs at tP; returns
-// sum(P). Masked elements get x = -inf, for which ex2 gives exactly 0.
-// With kWithMax it also reduces the half-row maximum of the raw scores alongside.
-// In unmasked tiles the pairs i (of 16 per 32 scores) with bit i of kEmu set take 2^x
-// from the FMA pipe (exp2_poly_f32x2) instead of the exp unit, so that the two pipes
-// share the exponentials.
-template <bool kMasked, bool kWithMax, uint32_t kEmu>
-__device__ __forceinline__ float softmax_half(uint32_t (&s)[2][32], uint32_t tP, float c,
-                                              float m_use, int climit, float* tile_max) {
-  float mx0 = -INFINITY, mx1 = -INFINITY;
-  uint64_t A01 = 0, A23 = 0;  // packed partial sums (+0.0f in both halves)
-  const uint64_t C2 = f2_pack(c, c);
-  const uint64_t NM2 = f2_pack(-m_use, -m_use);
-#pragma unroll
-  for (int q2 = 0; q2 < 2; ++q2) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float s0 = __uint_as_float(s[q2][2 * i]), s1 = __uint_as_float(s[q2][2 * i + 1]);
-      if (kWithMax) {
-        if (i & 1)
-          mx1 = fmax3(mx1, s0, s1);
-        else
-          mx0 = fmax3(mx0, s0, s1);
-      }
-      float x0, x1, e0, e1;
-      const uint64_t X = f2_fma(f2_pack(s0, s1), C2, NM2);
-      uint64_t E;
-      if (!kMasked && ((kEmu >> i) & 1u)) {
-        E = exp2_poly_f32x2(X);
-        f2_unpack(E, e0, e1);
-      } else {
-        f2_unpack(X, x0, x1);
-        if (kMasked) {
-          if (q2 * 32 + 2 * i > climit) x0 = -INFINITY;
-          if (q2 * 32 + 2 * i + 1 > climit) x1 = -INFINITY;
-        }
-        e0 = ex2_approx(x0);
-        e1 = ex2_approx(x1);
-        E = f2_pack(e0, e1);
-      }
-      if (i & 1)
-        A23 = f2_add(A23, E);
-      else
-        A01 = f2_add(A01, E);
-      pk[i] = pack_bf16x2(e0, e1);
-    }
-    tmem_st16(tP + q2 * 16, pk);
-  }
-  if (kWithMax) *tile_max = fmaxf(mx0, mx1);
-  float a0, a1, a2, a3;
-  f2_unpack(A01, a0, a1);
-  f2_unpack(A23, a2, a3);
-  return (a0 + a1) + (a2 + a3);
-}
-
 // One thread per row: 32 of the row's scores -> 16 columns of bf16 P pairs at tP, against
 // a known maximum (x = S * c - m); returns the sum of the 32 values of P. Masked elements
 // (index > climit) get x = -inf, for which ex2 gives exactly 0.
@@ -340,11 +259,11 @@ __device__ __forceinline__ float softmax_row32(const uint32_t (&s)[32], uint32_t
   return (a0 + a1) + (a2 + a3);
 }
 
-template <int D, bool kRow>
-__global__ void __launch_bounds__(FwdCfg<D, kRow>::kThreads, 1)
+template <int D>
+__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D, kRow>;
+  using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -352,8 +271,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
-  float* xch = reinterpret_cast<float*>(smem + C::kXchOff);
-  float* xl = reinterpret_cast<float*>(smem + C::kXlOff);
 
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int B_QF = 0, B_QE = 1;
@@ -491,9 +408,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint64_t dv0 = sdesc_sw128(sbase + C::kVOff, 16384, 1024);
         constexpr uint64_t kTileStep = C::kTileBytes >> 4;
 
-        // O_t += P_t V (stage vstage); acc=false overwrites O_t. Two threads per row:
-        // P_t's keys 0-63 sit in S_t columns [0,32), keys 64-127 in [64,96); one thread
-        // per row: keys 0-127 in columns [0,64).
+        // O_t += P_t V (stage vstage); acc=false overwrites O_t. P_t's keys 0-127 sit in
+        // S_t columns [0,64), 16 keys (8 columns) per MMA.
         auto issue_pv = [&](int t, int vstage, bool acc) {
           uint64_t dv = dv0 + (uint64_t)vstage * kTileStep;
           const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0);
@@ -501,8 +417,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           opaque(dv);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tO, tP + (kRow ? kk * 8 : (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8)),
-                   dv + (uint64_t)(kk * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+            mma_ts(tO, tP + kk * 8, dv + (uint64_t)(kk * 128), idesc_pv,
+                   (acc || kk > 0) ? 1u : 0u);
         };
         auto issue_qk = [&](int t, int kstage) {
           uint64_t dq = dq0 + (uint64_t)t * kTileStep;
@@ -574,471 +490,217 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else {
     regs_increase<C::kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax
-    if constexpr (!kRow) {
-      const int wg = warp / 4;
-      const int t = wg >> 1;                  // which Q tile of the unit
-      const int h = wg & 1;                   // which half of the 128 keys
-      const int wq = warp % 4;                // warp's TMEM lane quarter
-      const int r = wq * 32 + lane;           // row within the tile
-      const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0) + 64 * h;
-      const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0) + (D / 2) * h;
-      const uint32_t pair_bar = 1 + 4 * t + wq;  // the two warps that share these rows
-      float* xch_mine = xch + ((t * 2) * 2 + h) * 128 + r;        // + parity * 256
-      const float* xch_other = xch + ((t * 2) * 2 + (h ^ 1)) * 128 + r;
-      float* xl_mine = xl + (t * 2 + h) * 128 + r;
-      const float* xl_other = xl + (t * 2 + (h ^ 1)) * 128 + r;
-      const float c = p.scale_log2;
-      int scount = 0, ocount = 0;
-      bool ok = true;
-      // The two warps of a row pair meet at a named barrier once per key tile and once per
-      // epilogue. A warp that stops on an abort does one non-blocking arrival on its way
-      // out, which releases a partner already waiting; a partner not yet there sees the
-      // abort flag before the barrier and stops too.
-      auto pair_sync = [&]() -> bool {
-        if (*abort_flag) return false;
-        named_bar_sync(pair_bar, 64);
-        return true;
-      };
+    // one thread per row: thread r of softmax warpgroup t owns row r of Q tile t (TMEM
+    // lane r) and all 128 keys of each key tile; the tile maximum is known before any
+    // exponential, so P is computed once against the final base
+    const int t = warp / 4;                 // which Q tile of the unit
+    const int wq = warp % 4;                // warp's TMEM lane quarter
+    const int r = wq * 32 + lane;           // row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0);
+    const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0);
+    const float c = p.scale_log2;
+    int scount = 0, ocount = 0;
+    bool ok = true;
 
-      for (int rr = 0; ok; ++rr) {
-        const int u = unit_for_round(rr, blockIdx.x, G);
-        if (u >= n_units) break;
-        const Unit un = decode_unit(p, u);
-        const int qp = un.qp, bh = un.bh, n = un.n;
-        const PairDesc& pr = p.pair[un.pair];
-        const long long row0 = (long long)qp * 256 + t * 128;  // first row of this tile
-        const long long row = row0 + r;
-        const bool row_valid = row < pr.Nq;
-        // (the output addresses are formed where they are used, so that they are not
-        // held in registers through the key loop)
-        auto orow_of = [&]() { return pr.o + ((long long)bh * pr.Nq + row) * D + (D / 2) * h; };
-        auto lse_of = [&]() { return pr.lse + (long long)bh * pr.Nq + row; };
+    for (int rr = 0; ok; ++rr) {
+      const int u = unit_for_round(rr, blockIdx.x, G);
+      if (u >= n_units) break;
+      const Unit un = decode_unit(p, u);
+      const int qp = un.qp, bh = un.bh, n = un.n;
+      const PairDesc& pr = p.pair[un.pair];
+      const long long row0 = (long long)qp * 256 + t * 128;  // first row of this tile
+      const long long row = row0 + r;
+      const bool row_valid = row < pr.Nq;
+      auto orow_of = [&]() { return pr.o + ((long long)bh * pr.Nq + row) * D; };
+      auto lse_of = [&]() { return pr.lse + (long long)bh * pr.Nq + row; };
 
-        if (n == 0) {
-          // no key of this chunk is visible to the unit: the result is empty (O = 0,
-          // LSE = -inf), and folding an empty result into an accumulator changes nothing
-          if (row_valid && !p.accumulate) {
-            float4* o4 = reinterpret_cast<float4*>(orow_of());
-            for (int i = 0; i < D / 8; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (h == 0) *lse_of() = -INFINITY;
-          }
-          continue;
+      if (n == 0) {
+        // no key of this chunk is visible to the unit: the result is empty (O = 0,
+        // LSE = -inf), and folding an empty result into an accumulator changes nothing
+        if (row_valid && !p.accumulate) {
+          float4* o4 = reinterpret_cast<float4*>(orow_of());
+          for (int i = 0; i < D / 4; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          *lse_of() = -INFINITY;
         }
+        continue;
+      }
 
-        // last visible key index for this row (local to the chunk), and for the tile's
-        // first row (which decides whether a tile needs the per-element mask)
-        // (both in [-1, Nkv - 1], so they fit in int)
-        int lim_row = pr.Nkv - 1, lim_tile = pr.Nkv - 1;
-        if (p.causal) {
-          const long long a = pr.q_off + row - pr.kv_off, b = pr.q_off + row0 - pr.kv_off;
-          lim_row = a < lim_row ? (a < -1 ? -1 : (int)a) : lim_row;
-          lim_tile = b < lim_tile ? (b < -1 ? -1 : (int)b) : lim_tile;
-        }
+      // last visible key index for this row and for the tile's first row (both in
+      // [-1, Nkv - 1])
+      int lim_row = pr.Nkv - 1, lim_tile = pr.Nkv - 1;
+      if (p.causal) {
+        const long long a = pr.q_off + row - pr.kv_off, b = pr.q_off + row0 - pr.kv_off;
+        lim_row = a < lim_row ? (a < -1 ? -1 : (int)a) : lim_row;
+        lim_tile = b < lim_tile ? (b < -1 ? -1 : (int)b) : lim_tile;
+      }
 
-        float m = -INFINITY;  // running maximum (log2 units) used for the exponent
-        float l = 0.f;        // this half's running denominator
+      float m = -INFINITY;  // running maximum (log2 units) used for the exponent
+      float l = 0.f;        // running denominator
 
-        for (int j = 0; j < n; ++j) {
-          ok = mbar_wait(bar(B_SF + t), scount & 1, abort_flag, p.status);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          const int par = scount & 1;
-          ++scount;
-          tc_fence_after();
-
-          uint32_t s[2][32];
-          tmem_ld32(tS, s[0]);
-          tmem_ld32(tS + 32, s[1]);
-          tmem_ld_wait(s[0]);
-          reg_fence(s[1]);
-
-          const bool need_mask = (j * 128 + 127 > lim_tile);
-          // this half's keys with local column <= climit are visible for this row
-          const int cl = lim_row - (j * 128 + 64 * h);
-          const int climit = cl < -1 ? -1 : (cl > 63 ? 63 : cl);
-
-          float m_new, alpha, sum;
-          // both warps of a row pair take the same branch (same rows, same m)
-          if (__all_sync(0xffffffffu, !need_mask && m != -INFINITY)) {
-            // Common case: exponentiate against the current running maximum while the tile
-            // maximum is reduced alongside; the maximum only moves when a row's tile maximum
-            // exceeds it by more than 8 (log2 units). It then moves up by a whole number k
-            // of octaves (k >= the excess), so the P already stored only needs scaling by
-            // 2^-k, which is exact; P is recomputed only if it may have overflowed.
-            float mx;
-            sum = softmax_half<false, true, C::kEmu>(s, tS, c, m, climit, &mx);
-            xch_mine[par * 256] = mx;
-            if (!(ok = pair_sync())) break;
-            mx = fmaxf(mx, xch_other[par * 256]);
-            const float m_tile = mx * c;
-            const bool grow = m_tile > m + 8.0f;
-            m_new = m;
-            alpha = 1.f;
-            if (__any_sync(0xffffffffu, grow)) {
-              const float excess = m_tile - m;
-              const bool big = grow && excess > 100.0f;  // P against m may have overflowed
-              const int k = (grow && !big) ? (int)ceilf(excess) : 0;
-              m_new = grow ? (big ? m_tile : m + (float)k) : m;
-              alpha = big ? ex2_approx(m - m_new) : exp2_neg_int(k);
-              tmem_st_wait();  // the first P stores land before they are read back
-              if (__any_sync(0xffffffffu, big)) {
-                sum = softmax_half<false, false, C::kEmu>(s, tS, c, m_new, climit, nullptr);
-              } else {
-                const uint32_t a2 = pack_bf16x2(alpha, alpha);
-#pragma unroll 1
-                for (int q2 = 0; q2 < 2; ++q2) {  // rare: kept small rather than fast
-                  uint32_t pv[16];
-                  tmem_ld16(tS + q2 * 16, pv);
-                  tmem_ld_wait(pv);
-#pragma unroll
-                  for (int i = 0; i < 16; ++i) pv[i] = mul_bf16x2(pv[i], a2);
-                  tmem_st16(tS + q2 * 16, pv);
-                }
-                sum *= alpha;
-              }
-            }
-          } else {
-            float mx = -INFINITY;
-            {
-              float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float v0 = (2 * i > climit) ? -INFINITY : __uint_as_float(s[0][2 * i]);
-                const float v1 = (2 * i + 1 > climit) ? -INFINITY : __uint_as_float(s[0][2 * i + 1]);
-                const float v2 = (32 + 2 * i > climit) ? -INFINITY : __uint_as_float(s[1][2 * i]);
-                const float v3 =
-                    (33 + 2 * i > climit) ? -INFINITY : __uint_as_float(s[1][2 * i + 1]);
-                m0 = fmax3(m0, v0, v1);
-                m1 = fmax3(m1, v2, v3);
-              }
-              mx = fmaxf(m0, m1);
-            }
-            xch_mine[par * 256] = mx;
-            if (!(ok = pair_sync())) break;
-            mx = fmaxf(mx, xch_other[par * 256]);
-            const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * c;
-            m_new = (m_tile > m + 8.0f) ? m_tile : m;
-            // 1 when unchanged (also when both are -inf), 0 when m was -inf
-            alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            sum = need_mask ? softmax_half<true, false, 0u>(s, tS, c, m_use, climit, nullptr)
-                            : softmax_half<false, false, C::kEmu>(s, tS, c, m_use, climit, nullptr);
-          }
-          l = l * alpha + sum;
-
-          // rescale this thread's half of its row of O when its maximum moved
-          const bool moved = (m_new != m) && (j > 0);
-          if (__any_sync(0xffffffffu, moved)) {
-            const float a = moved ? alpha : 1.f;
-#pragma unroll
-            for (int q4 = 0; q4 < D / 64; ++q4) {
-              uint32_t ov[32];
-              tmem_ld32(tO + q4 * 32, ov);
-              tmem_ld_wait(ov);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * a);
-              tmem_st32(tO + q4 * 32, ov);
-            }
-          }
-          m = m_new;
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_PF + t));
-        }
-        if (!ok) break;
-
-        // ---------------------------------------------------------------- epilogue
-        ok = mbar_wait(bar(B_OD + t), ocount & 1, abort_flag, p.status);
+      for (int j = 0; j < n; ++j) {
+        ok = mbar_wait(bar(B_SF + t), scount & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        ++ocount;
+        ++scount;
         tc_fence_after();
-        // in accumulate mode both threads of the row read the old LSE before the pair
-        // barrier; the new one is written after it
-        float lse_acc = -INFINITY;
-        float* lse_row = lse_of();
-        if (p.accumulate && row_valid) lse_acc = *lse_row;
-        *xl_mine = l;
-        if (!(ok = pair_sync())) break;
-        const float l_row = l + *xl_other;
-        const bool nonempty = l_row > 0.f;
-        float lse_new = -INFINITY;
-        if (nonempty) {
-          float lg;
-          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l_row));
-          lse_new = (m + lg) * 0.69314718055994530942f;
-        }
-        // out = a * O_acc + b * O_tmem
-        float a = 0.f, b = nonempty ? 1.f / l_row : 0.f, lse_out = lse_new;
-        if (p.accumulate) {
-          const float M = fmaxf(lse_acc, lse_new);
-          if (M == -INFINITY) {
-            b = 0.f;
-          } else {
-            constexpr float kLog2e = 1.4426950408889634f;
-            const float wa = ex2_approx((lse_acc - M) * kLog2e);  // 0 for an empty accumulator
-            const float wn = ex2_approx((lse_new - M) * kLog2e);
-            const float inv = 1.f / (wa + wn);
-            a = wa * inv;
-            b = nonempty ? wn * inv / l_row : 0.f;
-            float lg;
-            asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(wa + wn));
-            lse_out = M + lg * 0.69314718055994530942f;
-          }
-        }
+
+        uint32_t s[4][32];
 #pragma unroll
-        for (int q4 = 0; q4 < D / 64; ++q4) {
-          uint32_t ov[32];
-          tmem_ld32(tO + q4 * 32, ov);
-          tmem_ld_wait(ov);
-          if (row_valid) {
-            float* dst = orow_of() + q4 * 32;
-            float res[32];
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, s[q]);
+        tmem_ld_wait(s[0]);
+        reg_fence(s[1]);
+        reg_fence(s[2]);
+        reg_fence(s[3]);
+
+        // the same for every row of the tile (it depends on the tile's first row)
+        const bool need_mask = (j * 128 + 127 > lim_tile);
+        const int cl = lim_row - j * 128;  // keys with local index <= climit are visible
+        const int climit = cl < -1 ? -1 : (cl > 127 ? 127 : cl);
+
+        // tile maximum of the raw scores over the visible keys (four partial maxima);
+        // two separate loops, so that unmasked tiles carry no per-element selects
+        float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (need_mask) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
-            if (a != 0.f) {  // only then is the old accumulator read
+          for (int q = 0; q < 4; ++q)
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 old = *reinterpret_cast<const float4*>(dst + i);
-                res[i] = fmaf(a, old.x, res[i]);
-                res[i + 1] = fmaf(a, old.y, res[i + 1]);
-                res[i + 2] = fmaf(a, old.z, res[i + 2]);
-                res[i + 3] = fmaf(a, old.w, res[i + 3]);
-              }
+            for (int i = 0; i < 16; ++i) {
+              const float v0 =
+                  (32 * q + 2 * i > climit) ? -INFINITY : __uint_as_float(s[q][2 * i]);
+              const float v1 =
+                  (32 * q + 2 * i + 1 > climit) ? -INFINITY : __uint_as_float(s[q][2 * i + 1]);
+              float& acc = mxa[(q & 1) * 2 + (i & 1)];
+              acc = fmax3(acc, v0, v1);
             }
-            if (p.o_vec8) {
+        } else {
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
-                             res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
-                             res[8 * i + 7]);
-            } else {
-              float4* o4 = reinterpret_cast<float4*>(dst);
+          for (int q = 0; q < 4; ++q)
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+            for (int i = 0; i < 16; ++i) {
+              float& acc = mxa[(q & 1) * 2 + (i & 1)];
+              acc = fmax3(acc, __uint_as_float(s[q][2 * i]), __uint_as_float(s[q][2 * i + 1]));
             }
-          }
         }
-        if (row_valid && h == 0) *lse_row = lse_out;
-        tc_fence_before();
-      }
-      if (!ok) named_bar_arrive(pair_bar, 64);
-    } else {
-      // one thread per row: thread r of softmax warpgroup t owns row r of Q tile t (TMEM
-      // lane r) and all 128 keys of each key tile; the tile maximum is known before any
-      // exponential, so P is computed once against the final base
-      const int t = warp / 4;                 // which Q tile of the unit
-      const int wq = warp % 4;                // warp's TMEM lane quarter
-      const int r = wq * 32 + lane;           // row within the tile
-      const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0);
-      const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0);
-      const float c = p.scale_log2;
-      int scount = 0, ocount = 0;
-      bool ok = true;
+        const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+        // The exponent base moves only when the tile maximum exceeds it by more than 8
+        // (log2 units), and then to the tile maximum: numerator and denominator share the
+        // base, so a stale one is exact, and P <= 2^8 stays well inside bf16 / fp32.
+        const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * c;
+        const float m_new = (m_tile > m + 8.0f) ? m_tile : m;
+        // 1 when unchanged (also when both are -inf), 0 when m was -inf
+        const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
 
-      for (int rr = 0; ok; ++rr) {
-        const int u = unit_for_round(rr, blockIdx.x, G);
-        if (u >= n_units) break;
-        const Unit un = decode_unit(p, u);
-        const int qp = un.qp, bh = un.bh, n = un.n;
-        const PairDesc& pr = p.pair[un.pair];
-        const long long row0 = (long long)qp * 256 + t * 128;  // first row of this tile
-        const long long row = row0 + r;
-        const bool row_valid = row < pr.Nq;
-        auto orow_of = [&]() { return pr.o + ((long long)bh * pr.Nq + row) * D; };
-        auto lse_of = [&]() { return pr.lse + (long long)bh * pr.Nq + row; };
-
-        if (n == 0) {
-          // no key of this chunk is visible to the unit: the result is empty (O = 0,
-          // LSE = -inf), and folding an empty result into an accumulator changes nothing
-          if (row_valid && !p.accumulate) {
-            float4* o4 = reinterpret_cast<float4*>(orow_of());
-            for (int i = 0; i < D / 4; ++i) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            *lse_of() = -INFINITY;
-          }
-          continue;
+        // P over S's first 64 columns (32 keys -> 16 columns): every score is in
+        // registers already
+        float sum;
+        if (need_mask) {
+          sum = softmax_row32<true, 0u>(s[0], tS, c, m_use, climit);
+          sum += softmax_row32<true, 0u>(s[1], tS + 16, c, m_use, climit - 32);
+          sum += softmax_row32<true, 0u>(s[2], tS + 32, c, m_use, climit - 64);
+          sum += softmax_row32<true, 0u>(s[3], tS + 48, c, m_use, climit - 96);
+        } else {
+          sum = softmax_row32<false, C::kEmu>(s[0], tS, c, m_use, 127);
+          sum += softmax_row32<false, C::kEmu>(s[1], tS + 16, c, m_use, 127);
+          sum += softmax_row32<false, C::kEmu>(s[2], tS + 32, c, m_use, 127);
+          sum += softmax_row32<false, C::kEmu>(s[3], tS + 48, c, m_use, 127);
         }
+        l = l * alpha + sum;
 
-        // last visible key index for this row and for the tile's first row (both in
-        // [-1, Nkv - 1])
-        int lim_row = pr.Nkv - 1, lim_tile = pr.Nkv - 1;
-        if (p.causal) {
-          const long long a = pr.q_off + row - pr.kv_off, b = pr.q_off + row0 - pr.kv_off;
-          lim_row = a < lim_row ? (a < -1 ? -1 : (int)a) : lim_row;
-          lim_tile = b < lim_tile ? (b < -1 ? -1 : (int)b) : lim_tile;
-        }
-
-        float m = -INFINITY;  // running maximum (log2 units) used for the exponent
-        float l = 0.f;        // running denominator
-
-        for (int j = 0; j < n; ++j) {
-          ok = mbar_wait(bar(B_SF + t), scount & 1, abort_flag, p.status);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ++scount;
-          tc_fence_after();
-
-          uint32_t s[4][32];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, s[q]);
-          tmem_ld_wait(s[0]);
-          reg_fence(s[1]);
-          reg_fence(s[2]);
-          reg_fence(s[3]);
-
-          // the same for every row of the tile (it depends on the tile's first row)
-          const bool need_mask = (j * 128 + 127 > lim_tile);
-          const int cl = lim_row - j * 128;  // keys with local index <= climit are visible
-          const int climit = cl < -1 ? -1 : (cl > 127 ? 127 : cl);
-
-          // tile maximum of the raw scores over the visible keys (four partial maxima);
-          // two separate loops, so that unmasked tiles carry no per-element selects
-          float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (need_mask) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float v0 =
-                    (32 * q + 2 * i > climit) ? -INFINITY : __uint_as_float(s[q][2 * i]);
-                const float v1 =
-                    (32 * q + 2 * i + 1 > climit) ? -INFINITY : __uint_as_float(s[q][2 * i + 1]);
-                float& acc = mxa[(q & 1) * 2 + (i & 1)];
-                acc = fmax3(acc, v0, v1);
-              }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                float& acc = mxa[(q & 1) * 2 + (i & 1)];
-                acc = fmax3(acc, __uint_as_float(s[q][2 * i]), __uint_as_float(s[q][2 * i + 1]));
-              }
-          }
-          const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
-          // The exponent base moves only when the tile maximum exceeds it by more than 8
-          // (log2 units), and then to the tile maximum: numerator and denominator share the
-          // base, so a stale one is exact, and P <= 2^8 stays well inside bf16 / fp32.
-          const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * c;
-          const float m_new = (m_tile > m + 8.0f) ? m_tile : m;
-          // 1 when unchanged (also when both are -inf), 0 when m was -inf
-          const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-
-          // P over S's first 64 columns (32 keys -> 16 columns): every score is in
-          // registers already
-          float sum;
-          if (need_mask) {
-            sum = softmax_row32<true, 0u>(s[0], tS, c, m_use, climit);
-            sum += softmax_row32<true, 0u>(s[1], tS + 16, c, m_use, climit - 32);
-            sum += softmax_row32<true, 0u>(s[2], tS + 32, c, m_use, climit - 64);
-            sum += softmax_row32<true, 0u>(s[3], tS + 48, c, m_use, climit - 96);
-          } else {
-            sum = softmax_row32<false, C::kEmu>(s[0], tS, c, m_use, 127);
-            sum += softmax_row32<false, C::kEmu>(s[1], tS + 16, c, m_use, 127);
-            sum += softmax_row32<false, C::kEmu>(s[2], tS + 32, c, m_use, 127);
-            sum += softmax_row32<false, C::kEmu>(s[3], tS + 48, c, m_use, 127);
-          }
-          l = l * alpha + sum;
-
-          // rescale this row of O when its base moved (P.V of the previous key tile has
-          // completed: the Q.K^T commit that released S follows it)
-          const bool moved = (m_new != m) && (j > 0);
-          if (__any_sync(0xffffffffu, moved)) {
-            const float a = moved ? alpha : 1.f;
+        // rescale this row of O when its base moved (P.V of the previous key tile has
+        // completed: the Q.K^T commit that released S follows it)
+        const bool moved = (m_new != m) && (j > 0);
+        if (__any_sync(0xffffffffu, moved)) {
+          const float a = moved ? alpha : 1.f;
 #pragma unroll 1
-            for (int q4 = 0; q4 < D / 32; ++q4) {
-              uint32_t ov[32];
-              tmem_ld32(tO + q4 * 32, ov);
-              tmem_ld_wait(ov);
+          for (int q4 = 0; q4 < D / 32; ++q4) {
+            uint32_t ov[32];
+            tmem_ld32(tO + q4 * 32, ov);
+            tmem_ld_wait(ov);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * a);
-              tmem_st32(tO + q4 * 32, ov);
-            }
-          }
-          m = m_new;
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_PF + t));
-        }
-        if (!ok) break;
-
-        // ---------------------------------------------------------------- epilogue
-        ok = mbar_wait(bar(B_OD + t), ocount & 1, abort_flag, p.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        ++ocount;
-        tc_fence_after();
-        float lse_acc = -INFINITY;
-        float* lse_row = lse_of();
-        if (p.accumulate && row_valid) lse_acc = *lse_row;
-        const bool nonempty = l > 0.f;
-        float lse_new = -INFINITY;
-        if (nonempty) {
-          float lg;
-          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
-          lse_new = (m + lg) * 0.69314718055994530942f;
-        }
-        // out = a * O_acc + b * O_tmem
-        float a = 0.f, b = nonempty ? 1.f / l : 0.f, lse_out = lse_new;
-        if (p.accumulate) {
-          const float M = fmaxf(lse_acc, lse_new);
-          if (M == -INFINITY) {
-            b = 0.f;
-          } else {
-            constexpr float kLog2e = 1.4426950408889634f;
-            const float wa = ex2_approx((lse_acc - M) * kLog2e);  // 0 for an empty accumulator
-            const float wn = ex2_approx((lse_new - M) * kLog2e);
-            const float inv = 1.f / (wa + wn);
-            a = wa * inv;
-            b = nonempty ? wn * inv / l : 0.f;
-            float lg;
-            asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(wa + wn));
-            lse_out = M + lg * 0.69314718055994530942f;
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * a);
+            tmem_st32(tO + q4 * 32, ov);
           }
         }
-#pragma unroll 1
-        for (int q4 = 0; q4 < D / 32; ++q4) {
-          uint32_t ov[32];
-          tmem_ld32(tO + q4 * 32, ov);
-          tmem_ld_wait(ov);
-          if (row_valid) {
-            float* dst = orow_of() + q4 * 32;
-            float res[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
-            if (a != 0.f) {  // only then is the old accumulator read
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 old = *reinterpret_cast<const float4*>(dst + i);
-                res[i] = fmaf(a, old.x, res[i]);
-                res[i + 1] = fmaf(a, old.y, res[i + 1]);
-                res[i + 2] = fmaf(a, old.z, res[i + 2]);
-                res[i + 3] = fmaf(a, old.w, res[i + 3]);
-              }
-            }
-            if (p.o_vec8) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
-                             res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
-                             res[8 * i + 7]);
-            } else {
-              float4* o4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
-            }
-          }
-        }
-        if (row_valid) *lse_row = lse_out;
+        m = m_new;
+        tmem_st_wait();
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PF + t));
       }
+      if (!ok) break;
+
+      // ---------------------------------------------------------------- epilogue
+      ok = mbar_wait(bar(B_OD + t), ocount & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++ocount;
+      tc_fence_after();
+      float lse_acc = -INFINITY;
+      float* lse_row = lse_of();
+      if (p.accumulate && row_valid) lse_acc = *lse_row;
+      const bool nonempty = l > 0.f;
+      float lse_new = -INFINITY;
+      if (nonempty) {
+        float lg;
+        asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
+        lse_new = (m + lg) * 0.69314718055994530942f;
+      }
+      // out = a * O_acc + b * O_tmem
+      float a = 0.f, b = nonempty ? 1.f / l : 0.f, lse_out = lse_new;
+      if (p.accumulate) {
+        const float M = fmaxf(lse_acc, lse_new);
+        if (M == -INFINITY) {
+          b = 0.f;
+        } else {
+          constexpr float kLog2e = 1.4426950408889634f;
+          const float wa = ex2_approx((lse_acc - M) * kLog2e);  // 0 for an empty accumulator
+          const float wn = ex2_approx((lse_new - M) * kLog2e);
+          const float inv = 1.f / (wa + wn);
+          a = wa * inv;
+          b = nonempty ? wn * inv / l : 0.f;
+          float lg;
+          asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(wa + wn));
+          lse_out = M + lg * 0.69314718055994530942f;
+        }
+      }
+#pragma unroll 1
+      for (int q4 = 0; q4 < D / 32; ++q4) {
+        uint32_t ov[32];
+        tmem_ld32(tO + q4 * 32, ov);
+        tmem_ld_wait(ov);
+        if (row_valid) {
+          float* dst = orow_of() + q4 * 32;
+          float res[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
+          if (a != 0.f) {  // only then is the old accumulator read
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 old = *reinterpret_cast<const float4*>(dst + i);
+              res[i] = fmaf(a, old.x, res[i]);
+              res[i + 1] = fmaf(a, old.y, res[i + 1]);
+              res[i + 2] = fmaf(a, old.z, res[i + 2]);
+              res[i + 3] = fmaf(a, old.w, res[i + 3]);
+            }
+          }
+          if (p.o_vec8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
+                           res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
+                           res[8 * i + 7]);
+          } else {
+            float4* o4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+          }
+        }
+      }
+      if (row_valid) *lse_row = lse_out;
+      tc_fence_before();
     }
   }
 

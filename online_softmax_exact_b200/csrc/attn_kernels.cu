@@ -55,12 +55,6 @@ __global__ void exp2_probe_kernel(const float* __restrict__ x, float* __restrict
 
 namespace {
 
-// softmax layout of the attention kernel (see FwdCfg): one thread per query row, or two
-#ifndef OSX_FWD_ROW
-#define OSX_FWD_ROW 1
-#endif
-constexpr bool kFwdRow = OSX_FWD_ROW != 0;
-
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
@@ -90,13 +84,13 @@ int device_info(DeviceInfo** out) {
         khz = 2000000;
       void* st = nullptr;
       if (cudaGetSymbolAddress(&st, g_device_status) != cudaSuccess) return ATTN_ERR_CUDA;
-      if (cudaFuncSetAttribute(attn_fwd_kernel<64, kFwdRow>,
+      if (cudaFuncSetAttribute(attn_fwd_kernel<64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)FwdCfg<64, kFwdRow>::kSmemBytes) != cudaSuccess)
+                               (int)FwdCfg<64>::kSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
-      if (cudaFuncSetAttribute(attn_fwd_kernel<128, kFwdRow>,
+      if (cudaFuncSetAttribute(attn_fwd_kernel<128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)FwdCfg<128, kFwdRow>::kSmemBytes) != cudaSuccess)
+                               (int)FwdCfg<128>::kSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
       di.num_sms = sms;
       di.clock_khz = khz;
@@ -172,8 +166,8 @@ int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) 
     p.unit_end[i] = static_cast<int>(units);
   }
   const int grid = units < di.num_sms ? static_cast<int>(units) : di.num_sms;
-  using Cfg = FwdCfg<D, kFwdRow>;
-  attn_fwd_kernel<D, kFwdRow><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
+  using Cfg = FwdCfg<D>;
+  attn_fwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return ATTN_OK;
