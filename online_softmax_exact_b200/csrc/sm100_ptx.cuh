@@ -156,16 +156,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Named barrier over `count` threads (a multiple of 32; id 0 is __syncthreads).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Arrive at a named barrier without waiting (releases peers that wait on it).
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // Register reallocation between warpgroups (all 128 threads of a warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void regs_increase() {
@@ -260,22 +250,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : OSX_R8(0), OSX_R8(8)
-      : "r"(taddr));
-}
-
 // Wait for this thread's outstanding tcgen05.ld; the registers passed are tied to the
 // wait so that no use of them can be scheduled before it.
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : OSX_RW8(0), OSX_RW8(8), OSX_RW8(16), OSX_RW8(24)::"memory");
-}
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" : OSX_RW8(0), OSX_RW8(8)::"memory");
 }
 // Tie further registers to an already-executed wait (keeps their uses after it).
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
@@ -321,17 +300,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
-
-// a * b for packed bf16 pairs (round to nearest; exact when b is a power of two and
-// the result stays normal)
-__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// 2^-k as a float, exactly, for an integer 0 <= k <= 126
-__device__ __forceinline__ float exp2_neg_int(int k) { return __int_as_float((127 - k) << 23); }
 
 // 256-bit global store of 8 floats (address 32-byte aligned)
 __device__ __forceinline__ void st_global_v8(float* p, float a0, float a1, float a2, float a3,
