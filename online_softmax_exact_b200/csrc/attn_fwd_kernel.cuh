@@ -14,7 +14,8 @@
 //     carries up to kMaxPairs pairs, their units in one static schedule;
 //   * warp 8 issues TMA loads (Q tiles once per unit, K and V tiles through rings of
 //     shared-memory stages, 128-byte swizzle);
-//   * warp 9 owns tensor memory and issues tcgen05.mma from one thread:
+//   * warp 9 owns tensor memory and issues tcgen05.mma (from lane 0 at D = 128; at
+//     D = 64 the whole warp runs the role in step and an elected lane issues):
 //     S_t = Q_t K_j^T (both operands in shared memory) into TMEM, then O_t += P_t V_j
 //     with P_t read from TMEM (written there by the softmax warps over S_t's columns);
 //   * two softmax warpgroups: warpgroup t owns Q tile t, one thread per query row (TMEM
@@ -81,11 +82,12 @@ struct FwdParams {
 
 // Pairs (bit i: pair i of every 16) of a thread's scores whose 2^x comes from the FMA
 // pipe in unmasked tiles, per head dimension. Measured on B200 (attn_fwd, TFLOP/s): at
-// D = 64, 4 pairs of 16 (25%) gain 1-2% over none; at D = 128 any share loses (the
+// D = 64, 6 pairs of 16 (37.5%, with the warp-wide MMA issue below) gain ~4% over 4
+// pairs issued from one lane, 8 pairs lose 15%; at D = 128 any share loses (the
 // polynomial's ~5 instructions per value, against 1, compete for issue slots with a
 // softmax that shares its tile period with twice the tensor work).
 #ifndef OSX_EMU_MASK_64
-#define OSX_EMU_MASK_64 0x2222u
+#define OSX_EMU_MASK_64 0x9249u
 #endif
 #ifndef OSX_EMU_MASK_128
 #define OSX_EMU_MASK_128 0x0000u
@@ -132,6 +134,11 @@ struct FwdCfg {
   static constexpr int kRegsOther = 72;
   // pairs of each 32-score block whose 2^x comes from the FMA pipe (bit i: pair i)
   static constexpr uint32_t kEmu = (D == 64) ? OSX_EMU_MASK_64 : OSX_EMU_MASK_128;
+  // MMA role run by the whole warp with elect.sync issue (D = 64), or by one lane
+  // (D = 128). Warp-wide issue shortens each tile's P.V + Q.K^T chain; the softmax
+  // warpgroups then overlap more, which at D = 128 costs more than the chain saves
+  // (measured 1-3% slower there) and at D = 64 gains 2-4% with the larger FMA share.
+  static constexpr bool kWarpIssue = (D == 64);
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 };
 
@@ -206,15 +213,18 @@ __device__ __forceinline__ int tail_rows_to_zero(const FwdParams& p, const Unit&
 // Zero rows [r0, 128) of a K/V tile in shared memory (D/64 boxes of 128 rows x 128
 // bytes; the 128-byte swizzle permutes 16-byte pieces within a row, so a row stays in
 // its own 128 bytes), then make the writes visible to the tensor core's operand reads.
-template <int D>
-__device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0) {
+// kLanes threads (1, or the 32 lanes of a warp, `lane` each) share the stores.
+template <int D, int kLanes>
+__device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0, int lane) {
 #pragma unroll 1
   for (int h = 0; h < D / 64; ++h) {
     const uint32_t end = tile + (h + 1) * 16384;
 #pragma unroll 4
-    for (uint32_t a = tile + h * 16384 + r0 * 128; a < end; a += 16) st_shared_zero16(a);
+    for (uint32_t a = tile + h * 16384 + r0 * 128 + lane * 16; a < end; a += 16 * kLanes)
+      st_shared_zero16(a);
   }
   fence_proxy_async_smem();
+  if (kLanes == 32) __syncwarp();
 }
 
 // One thread per row: 32 of the row's scores -> 16 columns of bf16 P pairs at tP, against
@@ -394,12 +404,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (warp == C::kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      // One lane, or the whole warp in step (every wait's outcome made uniform) with one
+      // elected lane issuing each tcgen05 instruction.
+      if (C::kWarpIssue || lane == 0) {
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
         int ks = 0, kph = 0, vs = 0, vph = 0, qcount = 0;
         int pv_steps = 0;  // P.V steps issued: both tiles' p_full barriers share its parity
         bool ok = true;
+        auto wait_u = [&](uint32_t b, int parity, volatile int* af, unsigned* st) -> bool {
+          const bool r = mbar_wait(b, parity, af, st);
+          if constexpr (C::kWarpIssue) return __all_sync(0xffffffffu, r);
+          return r;
+        };
+        auto commit = [&](uint32_t b) {
+          if constexpr (C::kWarpIssue) mma_commit_warp(b); else mma_commit(b);
+        };
         // Descriptors of the stage bases; the descriptor of (address + offset) is the
         // descriptor plus offset >> 4 (the start-address field is the low 14 bits and
         // every operand lies inside the CTA's shared memory window).
@@ -416,9 +436,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint32_t tP = tmem + (t ? C::kColS1 : C::kColS0);
           opaque(dv);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tO, tP + kk * 8, dv + (uint64_t)(kk * 128), idesc_pv,
-                   (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t b = dv + (uint64_t)(kk * 128);
+            const uint32_t en = (acc || kk > 0) ? 1u : 0u;
+            if constexpr (C::kWarpIssue)
+              mma_ts_warp(tO, tP + kk * 8, b, idesc_pv, en);
+            else
+              mma_ts(tO, tP + kk * 8, b, idesc_pv, en);
+          }
         };
         auto issue_qk = [&](int t, int kstage) {
           uint64_t dq = dq0 + (uint64_t)t * kTileStep;
@@ -429,7 +454,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)((kk / 4) * 1024 + (kk % 4) * 2);
-            mma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+            if constexpr (C::kWarpIssue)
+              mma_ss_warp(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
           }
         };
 
@@ -442,47 +470,49 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // V rows of the last key tile to zero before its P.V (the last of the unit)
           // reads them (128: none)
           const int vz_row = tail_rows_to_zero(p, un);
-          if (!(ok = mbar_wait(bar(B_QF), qcount & 1, abort_flag, p.status))) break;
+          if (!(ok = wait_u(bar(B_QF), qcount & 1, abort_flag, p.status))) break;
           ++qcount;
           tc_fence_after();
           for (int j = 0; j < n && ok; ++j) {
-            if (!(ok = mbar_wait(bar(B_KF + ks), kph, abort_flag, p.status))) break;
+            if (!(ok = wait_u(bar(B_KF + ks), kph, abort_flag, p.status))) break;
             tc_fence_after();
             for (int t = 0; t < 2; ++t) {
               if (j > 0) {
                 if (t == 0) {
-                  if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
+                  if (!(ok = wait_u(bar(B_VF + vs), vph, abort_flag, p.status))) break;
                 }
-                if (!(ok = mbar_wait(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
+                if (!(ok = wait_u(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
                 tc_fence_after();
                 issue_pv(t, vs, j > 1);
                 if (t == 1) {
                   ++pv_steps;
-                  mma_commit(bar(B_VE + vs));
+                  commit(bar(B_VE + vs));
                   if (++vs == C::kVStages) { vs = 0; vph ^= 1; }
                 }
               }
               issue_qk(t, ks);
-              mma_commit(bar(B_SF + t));
+              commit(bar(B_SF + t));
             }
             if (!ok) break;
-            mma_commit(bar(B_KE + ks));
+            commit(bar(B_KE + ks));
             if (++ks == C::kKStages) { ks = 0; kph ^= 1; }
           }
           if (!ok) break;
-          mma_commit(bar(B_QE));
+          commit(bar(B_QE));
           // last P.V of the unit
-          if (!(ok = mbar_wait(bar(B_VF + vs), vph, abort_flag, p.status))) break;
-          if (vz_row < 128) zero_tile_rows<D>(sbase + C::kVOff + vs * C::kTileBytes, vz_row);
+          if (!(ok = wait_u(bar(B_VF + vs), vph, abort_flag, p.status))) break;
+          if (vz_row < 128)
+            zero_tile_rows<D, C::kWarpIssue ? 32 : 1>(sbase + C::kVOff + vs * C::kTileBytes,
+                                                      vz_row, C::kWarpIssue ? lane : 0);
           for (int t = 0; t < 2; ++t) {
-            if (!(ok = mbar_wait(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
+            if (!(ok = wait_u(bar(B_PF + t), pv_steps & 1, abort_flag, p.status))) break;
             tc_fence_after();
             issue_pv(t, vs, n > 1);
-            mma_commit(bar(B_OD + t));
+            commit(bar(B_OD + t));
           }
           if (!ok) break;
           ++pv_steps;
-          mma_commit(bar(B_VE + vs));
+          commit(bar(B_VE + vs));
           if (++vs == C::kVStages) { vs = 0; vph ^= 1; }
         }
       }
@@ -711,8 +741,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (*abort_flag) {
     // let in-flight tensor-core work complete before TMEM is freed (the producer has
     // already waited for its copies)
-    if (warp == C::kWarpMma && lane == 0) {
-      mma_commit(bar(B_DRAIN));
+    if (warp == C::kWarpMma && (C::kWarpIssue || lane == 0)) {
+      // the commit comes from the issuer of the MMAs (the whole warp or lane 0)
+      if constexpr (C::kWarpIssue)
+        mma_commit_warp(bar(B_DRAIN));
+      else
+        mma_commit(bar(B_DRAIN));
       mbar_wait_drain(bar(B_DRAIN), 0, kDrainLimitNs);
     }
     __syncthreads();
