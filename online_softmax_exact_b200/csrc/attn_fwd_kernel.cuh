@@ -117,7 +117,15 @@ struct FwdCfg {
   // s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 6 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  // epilogue staging (D = 128): 32 rows x 32 fp32 (4 KB) per softmax warp, to turn each
+  // thread's row into coalesced 128-byte row segments. Measured on B200: +4% on the
+  // 128k GQA workload at D = 128, level elsewhere; at D = 64 it loses 5%, so D = 64
+  // stores each row from its own thread.
+  static constexpr bool kStagedEpilogue = (D == 128);
+  static constexpr uint32_t kStageOff = (kMiscOff + 16 + 1023) / 1024 * 1024;
+  static constexpr uint32_t kStageBytes = kStagedEpilogue ? 8 * 4096 : 0;
+  static constexpr uint32_t kSmemBytes = kStageOff + kStageBytes + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
   // warpgroups 0-1: softmax (tile t = warpgroup); warpgroup 2: {TMA producer, MMA
   // issuer, 2 idle}
   static constexpr int kThreads = 384;
@@ -695,37 +703,80 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           lse_out = M + lg * 0.69314718055994530942f;
         }
       }
-#pragma unroll 1
-      for (int q4 = 0; q4 < D / 32; ++q4) {
-        uint32_t ov[32];
-        tmem_ld32(tO + q4 * 32, ov);
-        tmem_ld_wait(ov);
-        if (row_valid) {
-          float* dst = orow_of() + q4 * 32;
-          float res[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
-          if (a != 0.f) {  // only then is the old accumulator read
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 old = *reinterpret_cast<const float4*>(dst + i);
-              res[i] = fmaf(a, old.x, res[i]);
-              res[i + 1] = fmaf(a, old.y, res[i + 1]);
-              res[i + 2] = fmaf(a, old.z, res[i + 2]);
-              res[i + 3] = fmaf(a, old.w, res[i + 3]);
+      if constexpr (C::kStagedEpilogue) {
+        // O in chunks of 32 columns: each thread scales its row's chunk and writes it to
+        // the warp's staging buffer (16-byte pieces XOR-swizzled by row, so that neither
+        // the row-wise writes nor the segment-wise reads conflict on banks); the warp then
+        // stores 4 rows' 128-byte segments per instruction (one thread per row would
+        // touch 32 lines per instruction). In accumulate mode the old values are read the
+        // same way and combined with the row's weight a.
+        float4* stage = reinterpret_cast<float4*>(smem + C::kStageOff + warp * 4096);
+        const int ch = lane & 7;
+  #pragma unroll 1
+        for (int q4 = 0; q4 < D / 32; ++q4) {
+          uint32_t ov[32];
+          tmem_ld32(tO + q4 * 32, ov);
+          tmem_ld_wait(ov);
+  #pragma unroll
+          for (int c = 0; c < 8; ++c)
+            stage[lane * 8 + (c ^ (lane & 7))] =
+                make_float4(__uint_as_float(ov[4 * c]) * b, __uint_as_float(ov[4 * c + 1]) * b,
+                            __uint_as_float(ov[4 * c + 2]) * b, __uint_as_float(ov[4 * c + 3]) * b);
+          __syncwarp();
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rl = i * 4 + (lane >> 3);  // row within the warp's 32
+            float4 v = stage[rl * 8 + (ch ^ (rl & 7))];
+            const float arow = __shfl_sync(0xffffffffu, a, rl);
+            const long long grow = row0 + wq * 32 + rl;
+            if (grow < pr.Nq) {
+              float* dst = pr.o + ((long long)bh * pr.Nq + grow) * D + q4 * 32 + ch * 4;
+              if (arow != 0.f) {  // only then is the old accumulator read
+                const float4 old = *reinterpret_cast<const float4*>(dst);
+                v.x = fmaf(arow, old.x, v.x);
+                v.y = fmaf(arow, old.y, v.y);
+                v.z = fmaf(arow, old.z, v.z);
+                v.w = fmaf(arow, old.w, v.w);
+              }
+              *reinterpret_cast<float4*>(dst) = v;
             }
           }
-          if (p.o_vec8) {
+          __syncwarp();  // the buffer is rewritten by the next chunk
+        }
+      } else {
+        // one thread per row: 32-byte stores of the row's own chunk
+#pragma unroll 1
+        for (int q4 = 0; q4 < D / 32; ++q4) {
+          uint32_t ov[32];
+          tmem_ld32(tO + q4 * 32, ov);
+          tmem_ld_wait(ov);
+          if (row_valid) {
+            float* dst = orow_of() + q4 * 32;
+            float res[32];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
-                           res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
-                           res[8 * i + 7]);
-          } else {
-            float4* o4 = reinterpret_cast<float4*>(dst);
+            for (int i = 0; i < 32; ++i) res[i] = __uint_as_float(ov[i]) * b;
+            if (a != 0.f) {  // only then is the old accumulator read
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+              for (int i = 0; i < 32; i += 4) {
+                const float4 old = *reinterpret_cast<const float4*>(dst + i);
+                res[i] = fmaf(a, old.x, res[i]);
+                res[i + 1] = fmaf(a, old.y, res[i + 1]);
+                res[i + 2] = fmaf(a, old.z, res[i + 2]);
+                res[i + 3] = fmaf(a, old.w, res[i + 3]);
+              }
+            }
+            if (p.o_vec8) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                st_global_v8(dst + 8 * i, res[8 * i], res[8 * i + 1], res[8 * i + 2],
+                             res[8 * i + 3], res[8 * i + 4], res[8 * i + 5], res[8 * i + 6],
+                             res[8 * i + 7]);
+            } else {
+              float4* o4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o4[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+            }
           }
         }
       }
