@@ -712,18 +712,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // same way and combined with the row's weight a.
         float4* stage = reinterpret_cast<float4*>(smem + C::kStageOff + warp * 4096);
         const int ch = lane & 7;
-  #pragma unroll 1
+#pragma unroll 1
         for (int q4 = 0; q4 < D / 32; ++q4) {
           uint32_t ov[32];
           tmem_ld32(tO + q4 * 32, ov);
           tmem_ld_wait(ov);
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 8; ++c)
             stage[lane * 8 + (c ^ (lane & 7))] =
                 make_float4(__uint_as_float(ov[4 * c]) * b, __uint_as_float(ov[4 * c + 1]) * b,
                             __uint_as_float(ov[4 * c + 2]) * b, __uint_as_float(ov[4 * c + 3]) * b);
           __syncwarp();
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int rl = i * 4 + (lane >> 3);  // row within the warp's 32
             float4 v = stage[rl * 8 + (ch ^ (rl & 7))];
