@@ -117,10 +117,11 @@ struct FwdCfg {
   // s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 6 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
-  // epilogue staging (D = 128): 32 rows x 32 fp32 (4 KB) per softmax warp, to turn each
-  // thread's row into coalesced 128-byte row segments. Measured on B200: +4% on the
-  // 128k GQA workload at D = 128, level elsewhere; at D = 64 it loses 5%, so D = 64
-  // stores each row from its own thread.
+  // epilogue staging (D = 128, outside accumulate mode): 32 rows x 32 fp32 (4 KB) per
+  // softmax warp, to turn each thread's row into coalesced 128-byte row segments.
+  // Measured on B200: +3-4% on the 128k GQA workload at D = 128, level elsewhere; at
+  // D = 64 it loses 5%, and the accumulating ring 4%, so those store each row from its
+  // own thread.
   static constexpr bool kStagedEpilogue = (D == 128);
   static constexpr uint32_t kStageOff = (kMiscOff + 16 + 1023) / 1024 * 1024;
   static constexpr uint32_t kStageBytes = kStagedEpilogue ? 8 * 4096 : 0;
@@ -703,13 +704,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           lse_out = M + lg * 0.69314718055994530942f;
         }
       }
-      if constexpr (C::kStagedEpilogue) {
+      if (C::kStagedEpilogue && !p.accumulate) {
         // O in chunks of 32 columns: each thread scales its row's chunk and writes it to
         // the warp's staging buffer (16-byte pieces XOR-swizzled by row, so that neither
         // the row-wise writes nor the segment-wise reads conflict on banks); the warp then
         // stores 4 rows' 128-byte segments per instruction (one thread per row would
-        // touch 32 lines per instruction). In accumulate mode the old values are read the
-        // same way and combined with the row's weight a.
+        // touch 32 lines per instruction). Accumulate mode, which also reads the old
+        // values, keeps one thread per row (measured faster there).
         float4* stage = reinterpret_cast<float4*>(smem + C::kStageOff + warp * 4096);
         const int ch = lane & 7;
 #pragma unroll 1
@@ -726,20 +727,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int rl = i * 4 + (lane >> 3);  // row within the warp's 32
-            float4 v = stage[rl * 8 + (ch ^ (rl & 7))];
-            const float arow = __shfl_sync(0xffffffffu, a, rl);
+            const float4 v = stage[rl * 8 + (ch ^ (rl & 7))];
             const long long grow = row0 + wq * 32 + rl;
-            if (grow < pr.Nq) {
-              float* dst = pr.o + ((long long)bh * pr.Nq + grow) * D + q4 * 32 + ch * 4;
-              if (arow != 0.f) {  // only then is the old accumulator read
-                const float4 old = *reinterpret_cast<const float4*>(dst);
-                v.x = fmaf(arow, old.x, v.x);
-                v.y = fmaf(arow, old.y, v.y);
-                v.z = fmaf(arow, old.z, v.z);
-                v.w = fmaf(arow, old.w, v.w);
-              }
-              *reinterpret_cast<float4*>(dst) = v;
-            }
+            if (grow < pr.Nq)
+              *reinterpret_cast<float4*>(pr.o + ((long long)bh * pr.Nq + grow) * D + q4 * 32 +
+                                         ch * 4) = v;
           }
           __syncwarp();  // the buffer is rewritten by the next chunk
         }
