@@ -26,9 +26,11 @@
 //     moved only when a tile maximum exceeds it by more than 8 (log2 units); exactness
 //     is kept because numerator and denominator share the same base. When m moves, the
 //     thread rescales its row of O in TMEM before releasing P;
-//   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32; in accumulate mode
-//     the result is first combined with the normalised partial (O_acc, LSE_acc) already
-//     in o/lse by the log-sum-exp rule of the merge (weights e^(LSE - max LSE)).
+//   * epilogue: O / l and LSE = (m + log2 l) ln 2, written as fp32 (at D = 128 through a
+//     per-warp shared-memory buffer, so that stores cover whole 128-byte row segments);
+//     in accumulate mode the result is first combined with the normalised partial
+//     (O_acc, LSE_acc) already in o/lse by the log-sum-exp rule of the merge (weights
+//     e^(LSE - max LSE)).
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [384,384+D). P_t (bf16 pairs, keys in order) overwrites S_t columns [0,64): a
