@@ -67,8 +67,11 @@ def test_accumulate_matches_the_merge_of_the_same_partials(osx):
             lse_ulps=MERGE_LSE_ULPS)
 
 
-def test_empty_accumulator_gives_the_plain_partial(osx):
-    q, k, v = inputs(2, 4, 2, 384, 384, 64, seed=9)
+@pytest.mark.parametrize("d", [64, 128])
+def test_empty_accumulator_gives_the_plain_partial(osx, d):
+    """At d = 128 the plain partial stores O through the shared-memory staging buffer and
+    the accumulating call stores it row by row: the two store paths must agree."""
+    q, k, v = inputs(2, 4, 2, 384, 384, d, seed=9)
     qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
     plain = osx.attn_fwd_partial(qg, kg, vg, q_start=0, q_len=384, kv_start=0, kv_len=384,
                                  causal=True)
