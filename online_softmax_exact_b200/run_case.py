@@ -2,10 +2,13 @@
 
     python -m online_softmax_exact_b200.run_case fwd   --B 1 --Hq 32 --N 8192 --d 128 [--causal]
     python -m online_softmax_exact_b200.run_case merge --parts 8 --rows 131072 --d 128
+    python -m online_softmax_exact_b200.run_case workload --name grid2d_64k_stress
 
 Does ``--warmup`` untimed calls then ``--reps`` timed calls (CUDA events on the
 launching stream) and prints one JSON line with the mean time and the achieved
-TFLOP/s (fwd) or GB/s (merge).
+TFLOP/s (fwd, workload) or GB/s (merge). ``workload`` runs one step of a named
+workload's schedule on its seeded inputs: the single pass, the ring's batched partials
+and merges, or the 2-D grid's batched cells and merges.
 """
 
 from __future__ import annotations
@@ -18,9 +21,36 @@ import torch
 import online_softmax_exact_b200 as osx
 
 
+def _workload_step(name: str, dev):
+    """(step callable, nominal FLOPs) of a named workload's schedule on its inputs."""
+    from workloads.configs import get
+    from workloads.gen import attention_inputs, grid_merge_orders
+
+    from . import schedules
+
+    w = get(name)
+    q, k, v = (t.to(dev) for t in attention_inputs(w))
+    if w.schedule == "ring":
+        ws = schedules.Workspace.for_shape(schedules.ring_slots(w.n_chunks, w.causal, True),
+                                           w.B, w.Hq, w.N // w.n_chunks, w.d, dev)
+        return (lambda: schedules.ring_attention(q, k, v, n_chunks=w.n_chunks, causal=w.causal,
+                                                 scale=w.scale, workspace=ws, batched=True),
+                w.flops)
+    if w.schedule == "grid2d":
+        P = w.n_chunks
+        ws = schedules.Workspace.for_shape(P * P, w.B, w.Hq, w.N // P, w.d, dev)
+        orders = grid_merge_orders(P, w.seed)
+        return (lambda: schedules.grid2d_attention(q, k, v, n_chunks=P, merge_orders=orders,
+                                                   causal=w.causal, scale=w.scale, workspace=ws,
+                                                   batched=True),
+                w.flops)
+    return (lambda: osx.attn_fwd(q, k, v, causal=w.causal, scale=w.scale), w.flops)
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["fwd", "merge"])
+    ap.add_argument("op", choices=["fwd", "merge", "workload"])
+    ap.add_argument("--name", default="grid2d_64k_stress")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--Hq", type=int, default=32)
     ap.add_argument("--Hkv", type=int, default=None)
@@ -45,6 +75,9 @@ def main(argv=None) -> int:
         lse = torch.empty((a.B, a.Hq, a.N), device=dev)
         run = lambda: osx.attn_fwd(q, k, v, causal=a.causal, o=o, lse=lse)  # noqa: E731
         work = 4.0 * a.B * a.Hq * a.N * a.N * a.d / (2 if a.causal else 1)
+        unit = "TFLOP/s"
+    elif a.op == "workload":
+        run, work = _workload_step(a.name, dev)
         unit = "TFLOP/s"
     else:
         op = [torch.randn((a.rows, a.d), device=dev, generator=g) for _ in range(a.parts)]
