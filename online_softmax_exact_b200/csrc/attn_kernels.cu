@@ -61,6 +61,7 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   int clock_khz = 0;           // peak SM clock
+  long long l2_bytes = 0;      // L2 cache size
   unsigned* status = nullptr;  // device address of g_device_status
 };
 
@@ -77,9 +78,11 @@ int device_info(DeviceInfo** out) {
   if (!di.ready) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!di.ready) {
-      int sms = 0, khz = 0;
+      int sms = 0, khz = 0, l2 = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return ATTN_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
+        l2 = 126 << 20;
       if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0)
         khz = 2000000;
       void* st = nullptr;
@@ -94,6 +97,7 @@ int device_info(DeviceInfo** out) {
         return ATTN_ERR_CUDA;
       di.num_sms = sms;
       di.clock_khz = khz;
+      di.l2_bytes = l2;
       di.status = static_cast<unsigned*>(st);
       di.ready = true;
     }
@@ -105,6 +109,33 @@ int device_info(DeviceInfo** out) {
 // three tensor maps plus the parameter block stay within the classic 4 KB of kernel
 // parameters
 static_assert(3 * sizeof(CUtensorMap) + sizeof(FwdParams) <= 4096, "kernel parameters");
+
+// Key tiles that one (batch, head) of a pair visits over all its 256-row blocks, and the
+// most that one block visits.
+double pair_tiles(const PairLaunch& s, int causal) {
+  const long long tiles = (s.kv_len + 127) / 128;
+  const long long nqp = (s.q_len + 255) / 256;
+  if (!causal) return (double)tiles * nqp;
+  double sum = 0.0;
+  for (long long qp = 0; qp < nqp; ++qp) {
+    long long last = qp * 256 + 255;
+    if (last > s.q_len - 1) last = s.q_len - 1;
+    const long long lim = s.q_off + last - s.kv_off;
+    if (lim < 0) continue;
+    const long long n = lim / 128 + 1;
+    sum += (double)(n < tiles ? n : tiles);
+  }
+  return sum;
+}
+
+long long heaviest_unit_tiles(const PairLaunch& s, int causal) {
+  const long long tiles = (s.kv_len + 127) / 128;
+  if (!causal) return tiles;
+  const long long lim = s.q_off + s.q_len - 1 - s.kv_off;
+  if (lim < 0) return 0;
+  const long long n = lim / 128 + 1;
+  return n < tiles ? n : tiles;
+}
 
 template <int D>
 int launch_fwd_d(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) {
@@ -194,15 +225,83 @@ int launch_merge_d(const MergeParams& p, const DeviceInfo& di, cudaStream_t stre
 
 }  // namespace
 
+namespace {
+
+int launch_fwd_one(const FwdLaunch& a, const DeviceInfo& di, cudaStream_t stream) {
+  switch (a.d) {
+    case 64: return launch_fwd_d<64>(a, di, stream);
+    case 128: return launch_fwd_d<128>(a, di, stream);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+// Key/value heads per launch for a one-pair call with a causal cut whose K/V (all heads)
+// exceed three quarters of L2: the fewest whose K/V fit in three quarters of L2 while the
+// launch's heaviest work unit stays within a fifth of a CTA's share of it; 0: one launch.
+// The kernel runs a pair's units row block by row block, heaviest first, all heads side by
+// side; once the CTAs drift apart they stream different heads' K/V at different key
+// positions, and K/V that do not fit in L2 are then read from DRAM many times over
+// (measured on B200 for the 128k GQA workload: 203 GB of reads for 0.54 GB of K/V).
+// Launching a few key/value heads at a time keeps the K/V being read within L2.
+int kv_heads_per_launch(const FwdLaunch& a, const DeviceInfo& di) {
+  if (a.n_pairs != 1 || !a.causal) return 0;
+  const PairLaunch& s = a.pairs[0];
+  const double kv_head_bytes = (double)s.kv_len * a.d * 4.0;  // K and V of one head
+  const double budget = 0.75 * (double)di.l2_bytes;
+  if (kv_head_bytes * a.B * a.Hkv <= budget) return 0;
+  {
+    // no causal cut inside the pair (even its first row block sees every key tile): the
+    // kernel runs such pairs head by head already
+    const long long kv_tiles = (s.kv_len + 127) / 128;
+    const long long last_row0 = (s.q_len < 256 ? s.q_len : 256) - 1;
+    if (s.q_off + last_row0 - s.kv_off >= (kv_tiles - 1) * 128) return 0;
+  }
+  const double tiles = pair_tiles(s, a.causal);  // one head's key tiles over all units
+  const double heaviest = (double)heaviest_unit_tiles(s, a.causal);
+  const int group = a.Hq / a.Hkv;
+  const long long qp = (s.q_len + 255) / 256;
+  for (int k = 1; k < a.Hkv; ++k) {
+    if (a.Hkv % k != 0) continue;
+    if (k * kv_head_bytes > budget) break;
+    const long long units = qp * k * group;
+    const double ctas = (double)(units < di.num_sms ? units : di.num_sms);
+    if (heaviest <= 0.2 * tiles * k * group / ctas) return k;
+  }
+  return 0;
+}
+
+}  // namespace
+
 int launch_fwd(const FwdLaunch& a, cudaStream_t stream) {
   DeviceInfo* di = nullptr;
   int rc = device_info(&di);
   if (rc != ATTN_OK) return rc;
-  switch (a.d) {
-    case 64: return launch_fwd_d<64>(a, *di, stream);
-    case 128: return launch_fwd_d<128>(a, *di, stream);
-    default: return ATTN_ERR_UNSUPPORTED;
+  const int k = kv_heads_per_launch(a, *di);
+  if (k == 0) return launch_fwd_one(a, *di, stream);
+  // the same pair over bands of k key/value heads (and their query heads), one launch
+  // each: every band's rows of Q, K, V, O and LSE are contiguous
+  const int group = a.Hq / a.Hkv;
+  const PairLaunch& s = a.pairs[0];
+  for (int b = 0; b < a.B; ++b) {
+    for (int g = 0; g < a.Hkv; g += k) {
+      const long long qh = (long long)b * a.Hq + (long long)g * group;  // first query head
+      const long long kvh = (long long)b * a.Hkv + g;                  // first K/V head
+      PairLaunch pr = s;
+      pr.o = s.o + qh * s.q_len * a.d;
+      pr.lse = s.lse + qh * s.q_len;
+      FwdLaunch band = a;
+      band.q = static_cast<const char*>(a.q) + qh * a.q_ld * a.d * 2;
+      band.k = static_cast<const char*>(a.k) + kvh * a.kv_ld * a.d * 2;
+      band.v = static_cast<const char*>(a.v) + kvh * a.kv_ld * a.d * 2;
+      band.B = 1;
+      band.Hq = k * group;
+      band.Hkv = k;
+      band.pairs = &pr;
+      rc = launch_fwd_one(band, *di, stream);
+      if (rc != ATTN_OK) return rc;
+    }
   }
+  return ATTN_OK;
 }
 
 int launch_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts,
