@@ -89,3 +89,38 @@ def test_grid2d_64k_stress(osx):
             assert osx.attn_device_status() == osx.ATTN_OK
             o, lse = chunks_to_sequence(oc, lc)
             check_sampled(o, lse, q, k, v, w, 96 if batched and not fused else 32)
+
+
+def test_large_causal_gqa_over_key_value_head_bands(osx):
+    """A one-pair causal call whose K/V exceed L2 is launched over bands of key/value
+    heads (here B = 2, 8 key/value heads of 4 query heads, N = 65536: two key/value heads
+    per launch, eight launches). Every band's O and LSE rows, in both batches, must equal
+    the oracle's; a partial on a chunk of the parents with global offsets, folded into an
+    accumulator, goes the same way."""
+    from workloads.gen import randn_bf16
+
+    B, Hq, Hkv, N, d = 2, 32, 8, 65536, 128
+    q = randn_bf16((B, Hq, N, d), 21, 0)
+    k = randn_bf16((B, Hkv, N, d), 21, 1)
+    v = randn_bf16((B, Hkv, N, d), 21, 2)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    scale = d ** -0.5
+    launches = osx.attn_launch_count()
+    o, lse = osx.attn_fwd(qg, kg, vg, causal=True, scale=scale)
+    assert osx.attn_device_status() == osx.ATTN_OK
+    assert osx.attn_launch_count() - launches == 8
+    rows = sample_rows(N, 16384, 40, seed=21)
+    rows_t = torch.from_numpy(rows).cuda()
+    o_ref, l_ref = oracle.attention_rows(q, k, v, causal=True, scale=scale, rows=rows)
+    do, dl = compare(to_np(o.index_select(2, rows_t)), to_np(lse.index_select(2, rows_t)),
+                     o_ref, l_ref)
+    print(f"banded GQA B=2: {len(rows)} rows/head, max|dO|={do:.2e} max|dLSE|={dl:.2e}")
+    # the second half of the keys folded into the first half's partial: the whole result
+    h = N // 2
+    acc_o, acc_l = osx.attn_fwd_partial(qg, kg, vg, q_start=0, q_len=N, kv_start=0, kv_len=h,
+                                        causal=True, scale=scale)
+    osx.attn_fwd_partial_acc(qg, kg, vg, q_start=0, q_len=N, kv_start=h, kv_len=h,
+                             causal=True, scale=scale, o=acc_o, lse=acc_l)
+    assert osx.attn_device_status() == osx.ATTN_OK
+    compare(to_np(acc_o.index_select(2, rows_t)), to_np(acc_l.index_select(2, rows_t)),
+            o_ref, l_ref)
